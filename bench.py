@@ -1,0 +1,386 @@
+"""Benchmark of the RRAttention prefill hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama128k] [--impl reference]
+
+One step = one attention layer's prefill: pooled-key estimate, Top-tau select and block-sparse
+attention (rra_estimate, rra_select, rra_sparse_attn through the C ABI) on the seeded
+Llama-3.1-8B-like layer at 128K tokens (b1, 32 Q / 8 KV heads, d 128, B 128, S 8, tau 0.9).
+Inputs (2.7 GB) are larger than L2, so no flush is needed between steps. With N > 1 (torchrun)
+every rank runs an independent replica of the layer; the time is the max over ranks.
+
+Prints one JSON line (rank 0). `value` is milliseconds per layer for the whole job
+(max-over-ranks step time / layers processed per step). The reference arm times the fp64 CPU
+oracle on a bounded sample of block rows of the same workload and extrapolates to a layer.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+from long_context_prefill_rr_b200 import workloads as wl  # noqa: E402
+
+METRIC = "prefill attn ms/layer @128K (estimate+select+sparse) & TFLOP/s vs roofline"
+UNIT = "ms/layer"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d["bf16_tflops_sustained"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1590.0,
+            "source": "fallback"}
+
+
+def _workload_desc(w: wl.Workload) -> dict:
+    return {"workload": f"{w.name}: b{w.batch} Hq{w.heads_q} Hkv{w.heads_kv} d{w.head_dim} "
+                        f"L{w.seqlen} B{w.block} S{w.stride} tau{w.tau}",
+            "model": "Llama-3.1-8B-like attention layer (random synthetic Q/K/V)"
+            if w.kind == "llama" else w.kind,
+            "global_batch": w.batch, "seq_len": w.seqlen, "heads_q": w.heads_q,
+            "heads_kv": w.heads_kv, "head_dim": w.head_dim, "block": w.block, "stride": w.stride,
+            "tau": w.tau, "parallelism": "replicas", "l2": "inputs (2.7 GB) larger than L2"
+            if w.seqlen >= 32768 else "L2 flushed between steps"}
+
+
+def attention_flops(kept_idx: np.ndarray, kept_cnt: np.ndarray, block: int, d: int):
+    """(useful, executed) flops of the block-sparse attention: 2 GEMMs x 2 flops per MAC;
+    useful counts only the causal half (B(B+1)/2 pairs) of diagonal blocks."""
+    b, h, nb = kept_cnt.shape
+    n_kept = int(kept_cnt.sum(dtype=np.int64))
+    n_diag = 0
+    for I in range(nb):
+        off = I * (I + 1) // 2
+        cnt = kept_cnt[:, :, I]
+        last = kept_idx[:, :, off:off + I + 1]
+        # the diagonal, if kept, is the last entry of the ascending row
+        pos = np.clip(cnt - 1, 0, None)
+        lastv = np.take_along_axis(last, pos[..., None], axis=2)[..., 0]
+        n_diag += int(((cnt > 0) & (lastv == I)).sum())
+    useful = 4.0 * d * (block * block * (n_kept - n_diag) + block * (block + 1) / 2 * n_diag)
+    executed = 4.0 * d * block * block * n_kept
+    return useful, executed, n_kept
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self) -> dict:
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_oracle_sample(w: wl.Workload, q_bits, k_bits, v_bits, n_rows: int, seed: int = 0,
+                      total_kept: int | None = None) -> dict:
+    """Time the fp64 oracle (estimate -> select -> attention, each on the oracle's own outputs)
+    on a seeded sample of block rows and extrapolate to one layer.
+
+    Estimate and select cost scale with the row length (I + 1 blocks), attention with the
+    row's kept blocks; each phase's per-unit time from the sample is multiplied by the layer's
+    total units (total kept blocks: ``total_kept`` when known, else the sample's kept fraction
+    times every causal block).
+    """
+    import oracle as orc
+    scale = w.softmax_scale if w.softmax_scale > 0 else 1.0 / np.sqrt(w.head_dim)
+    nb = w.seqlen // w.block
+    rng = np.random.default_rng(seed)
+    rows = [(0, int(rng.integers(w.heads_q)), int(rng.integers(nb))) for _ in range(n_rows)]
+    t_est = t_att = 0.0
+    u_est = u_att = 0
+    kbars = {}
+    t0 = time.perf_counter()
+    for b, h, I in rows:
+        kv = orc.kv_head(h, w.heads_q, w.heads_kv)
+        q = wl.bf16_bits_to_f64(q_bits[b, h])
+        k = wl.bf16_bits_to_f64(k_bits[b, kv])
+        v = wl.bf16_bits_to_f64(v_bits[b, kv])
+        a = time.perf_counter()
+        if (b, kv) not in kbars:
+            kbars[(b, kv)] = orc.pooled_keys(k, w.stride)
+        mass = orc.estimate_block_row(q, kbars[(b, kv)], h, I, w.block, w.stride, w.shift, scale)
+        kept = orc.select_row(mass, I, w.tau)
+        c = time.perf_counter()
+        orc.attention_block(q, k, v, I, kept, w.block, scale)
+        e = time.perf_counter()
+        t_est += c - a
+        t_att += e - c
+        u_est += I + 1
+        u_att += len(kept)
+    wall = time.perf_counter() - t0
+    total_causal = w.batch * w.heads_q * nb * (nb + 1) // 2
+    if total_kept is None:
+        total_kept = u_att / u_est * total_causal
+        how = "the sample's kept fraction"
+    else:
+        how = "the GPU run's kept-block count"
+    ms = 1e3 * (t_est / u_est * total_causal + t_att / max(u_att, 1) * total_kept)
+    return {"value": ms, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+            "sample": f"{n_rows} seeded (head, block-row) pairs of {w.name}, fp64 numpy "
+                      f"({wall:.1f} s), extrapolated to the layer by row length (estimate + "
+                      f"select) and kept blocks (attention; total from {how})",
+            "sample_seconds": wall}
+
+
+def _dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def run_reference(args, w):
+    ws, rank, _ = _dist_env()
+    if rank != 0:
+        return 0
+    q_bits, k_bits, v_bits = wl.make_workload(w)
+    step_ms = []
+    cb = None
+    for s in range(args.warmup + args.steps):
+        cb = cpu_oracle_sample(w, q_bits, k_bits, v_bits, n_rows=args.ref_rows, seed=s)
+        if s >= args.warmup:
+            step_ms.append(cb["value"])
+    value = float(np.mean(step_ms))
+    cb["value"] = value
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": value, "higher_is_better": False,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": _workload_desc(w), "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_gpu(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from long_context_prefill_rr_b200 import native
+
+    ws_n, rank, local = _dist_env()
+    if ws_n > 1:
+        dist.init_process_group("nccl", init_method="env://",
+                                timeout=__import__("datetime").timedelta(seconds=600))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    native.load()
+    p = native.params(w.batch, w.heads_q, w.heads_kv, w.seqlen, w.head_dim, w.stride, w.tau,
+                      shift=w.shift, softmax_scale=w.softmax_scale, block=w.block)
+    sh = native.shapes(p)
+    q_bits, k_bits, v_bits = wl.make_workload(w)
+
+    def host_pinned(bits):
+        t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory()
+
+    hq, hk, hv = host_pinned(q_bits), host_pinned(k_bits), host_pinned(v_bits)
+    q = hq.to(dev)
+    k = hk.to(dev)
+    v = hv.to(dev)
+    out = torch.empty(sh["q"], dtype=torch.bfloat16, device=dev)
+    mass = torch.empty(sh["mass"], dtype=torch.float32, device=dev)
+    idx = torch.empty(sh["kept_idx"], dtype=torch.int32, device=dev)
+    cnt = torch.empty(sh["kept_cnt"], dtype=torch.int32, device=dev)
+    wsp = native.new_workspace(p, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        native.estimate(p, q, k, mass, wsp)
+        if ev is not None:
+            ev[1].record(stream)
+        native.select(p, mass, idx, cnt)
+        if ev is not None:
+            ev[2].record(stream)
+        native.sparse_attn(p, q, k, v, idx, cnt, out, wsp)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    st, raw = native.check_device_status(wsp)
+    if st != 0:
+        raise RuntimeError(f"device status {raw:#x} after warm-up")
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws_n > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        start.record(stream)
+        for s in range(args.steps):
+            step(events[s])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if ws_n > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    est_ms = [e[0].elapsed_time(e[1]) for e in events]
+    sel_ms = [e[1].elapsed_time(e[2]) for e in events]
+    att_ms = [e[2].elapsed_time(e[3]) for e in events]
+    st, raw = native.check_device_status(wsp)
+    if st != 0:
+        raise RuntimeError(f"device status {raw:#x} after the timed steps")
+
+    # ---- end to end through the public one-call API with host buffers
+    hout = torch.empty(sh["q"], dtype=torch.bfloat16).pin_memory()
+    e_start, e_stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_steps = max(1, min(args.steps, 5))
+    torch.cuda.synchronize(dev)
+    e_start.record(stream)
+    for _ in range(e_steps):
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        native.prefill(p, q, k, v, out, idx, cnt, wsp, mass=mass)
+        hout.copy_(out, non_blocking=True)
+    e_stop.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e_start.elapsed_time(e_stop) / e_steps
+
+    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+    if ws_n > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    if rank == 0:
+        peaks = _peaks()
+        kept_idx = idx.cpu().numpy()
+        kept_cnt = cnt.cpu().numpy()
+        useful, executed, n_kept = attention_flops(kept_idx, kept_cnt, w.block, w.head_dim)
+        nb = w.seqlen // w.block
+        density = n_kept / (w.batch * w.heads_q * nb * (nb + 1) / 2)
+        att_avg = float(np.mean(att_ms))
+        est_avg = float(np.mean(est_ms))
+        sel_avg = float(np.mean(sel_ms))
+        achieved = useful / (att_avg * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        ns = w.seqlen // w.stride
+        est_bytes = (w.batch * w.heads_kv * w.seqlen * w.head_dim * 2          # K read once
+                     + w.batch * w.heads_q * ns * w.head_dim * 2               # sampled Q rows
+                     + w.batch * w.heads_q * nb * (nb + 1) // 2 * 4)           # masses out
+        sel_bytes = (w.batch * w.heads_q * nb * (nb + 1) // 2 * 4 + n_kept * 4 +
+                     w.batch * w.heads_q * nb * 4)
+        ms_per_step = total_ms / args.steps
+        value = ms_per_step / ws_n
+        cpu = None
+        if ws_n == 1 and not args.no_cpu_baseline:
+            cpu = cpu_oracle_sample(w, q_bits, k_bits, v_bits, n_rows=args.ref_rows,
+                                    total_kept=n_kept)
+        traffic = None
+        tpath = os.path.join(ROOT, "profiles", "attn_traffic.json")
+        if os.path.exists(tpath):
+            td = json.load(open(tpath))
+            if td.get("workload") == w.name and td.get("kernel_rev") == KERNEL_REV:
+                traffic = td.get("bytes_per_launch")
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, shaped like the pages' Llama-3.1-8B 128K workload)",
+            "config": _workload_desc(w),
+            "phases_ms": {"estimate": est_avg, "select": sel_avg, "sparse_attn": att_avg},
+            "density": density,
+            "attn_tflops": achieved, "attn_tflops_executed": executed / (att_avg * 1e-3) / 1e12,
+            "estimate_gbs": est_bytes / (est_avg * 1e-3) / 1e9,
+            "estimate_frac_hbm": est_bytes / (est_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "select_gbs": sel_bytes / (sel_avg * 1e-3) / 1e9,
+            "estimate_select_frac_hbm": (est_bytes + sel_bytes) / ((est_avg + sel_avg) * 1e-3)
+            / 1e9 / peaks["hbm_gbs"],
+            "roofline": {"bound": "tensor", "kernel": "bs_attn_fwd_kernel", "achieved": achieved,
+                         "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{peaks['source']} bf16 sustained",
+                         "traffic": traffic,
+                         "per_launch_flops": useful},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_ms / ws_n, "unit": UNIT,
+                    "h2d_bytes_per_step": int(hq.numel() + hk.numel() + hv.numel()) * 2,
+                    "d2h_bytes_per_step": int(hout.numel()) * 2},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# bump when the attention kernel changes, so stale ncu traffic is not reported
+KERNEL_REV = "attn-v1"
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama128k", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=12)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    w = wl.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,120 @@
+/*
+ * rra.h - C ABI of the RRAttention prefill hot path on NVIDIA B200 (sm_100a).
+ *
+ * The path (RRAttention: "Dynamic Block Sparse Attention via Per-Head Round-Robin Shifts for
+ * Long-Context Inference", abstract; and the research summary of the same paper, "Summary" and
+ * "Key points"):
+ *
+ *   1. estimate  - in every stride of S tokens head h scores the one query at in-stride offset
+ *                  (h + shift) mod S against the stride-summed keys, takes a causal softmax over
+ *                  the stride-level scores, and sums the probabilities into B x B blocks.
+ *   2. select    - per head and query-block row keep the smallest set of key blocks whose mass
+ *                  reaches tau (the find_blocks rule of the XAttention review, section 3), plus
+ *                  the diagonal block.
+ *   3. attention - causal block-sparse attention over the kept blocks (GQA, online softmax).
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are row-major and contiguous: Q [batch, heads_q, seqlen, head_dim],
+ *     K and V [batch, heads_kv, seqlen, head_dim], O like Q; all bf16.
+ *   - GQA: query head h reads KV head h / (heads_q / heads_kv).
+ *   - Block masses `mass` (fp32) and kept lists `kept_idx` (int32) are packed lower triangles,
+ *     one per (batch, head): block row I occupies entries [I(I+1)/2, I(I+1)/2 + I + 1), entry J
+ *     belongs to key block J. NB = seqlen / block rows; NB(NB+1)/2 entries per (batch, head).
+ *     A kept row lists its key blocks in ascending order; unused entries hold -1.
+ *     `kept_cnt` int32 [batch, heads_q, NB] is the length of each kept row.
+ *   - Each estimated block row sums to 1: mass(I, J) = (1/m) sum over the m = block/stride
+ *     sampled queries i of row I of the stride-softmax probabilities of the strides in block J.
+ *   - All pointers are DEVICE pointers, 16-byte aligned, owned by the caller. The library never
+ *     allocates or frees memory; all work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns without synchronising, except rra_check_device_status.
+ *   - Argument errors are reported before anything is enqueued. A failed launch returns
+ *     RRA_ERR_CUDA. Kernels never trap: a device-side wait that exceeds its time limit, or an
+ *     invalid kept list met by the attention kernel, sets a sticky error word in the workspace,
+ *     which rra_check_device_status reads and clears.
+ *   - An empty problem (batch == 0 or seqlen == 0) is valid and enqueues nothing.
+ */
+#ifndef RRA_H_
+#define RRA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RRA_OK = 0,
+  RRA_ERR_INVALID_ARG = 1,    /* null/misaligned pointer, inconsistent shape, bad tau, bad list */
+  RRA_ERR_UNSUPPORTED = 2,    /* valid but not implemented: block != 128, head_dim, stride */
+  RRA_ERR_WORKSPACE = 3,      /* workspace smaller than rra_workspace_bytes() */
+  RRA_ERR_CUDA = 4,           /* a CUDA runtime / driver call failed */
+  RRA_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up waiting on a barrier (see status word) */
+} rra_status;
+
+typedef struct {
+  int batch;          /* b >= 0 */
+  int heads_q;        /* Hq >= 1 */
+  int heads_kv;       /* Hkv >= 1, Hq % Hkv == 0 */
+  int seqlen;         /* L >= 0, L % block == 0 */
+  int head_dim;       /* d in {64, 128} */
+  int block;          /* B; 128 is the only supported block size */
+  int stride;         /* S in {4, 8, 16, 32}; must divide B */
+  int shift;          /* round-robin shift; any integer, reduced mod S */
+  float tau;          /* (0, 1]; tau >= 1 keeps every causal block */
+  float softmax_scale;/* applied to q.k in both the estimate and the attention; <= 0 means
+                         1/sqrt(head_dim) */
+} rra_params;
+
+typedef struct CUstream_st *rra_stream_t;   /* same type as cudaStream_t */
+
+/* Bytes of device workspace needed by rra_estimate / rra_sparse_attn / rra_prefill for these
+ * parameters on the CURRENT device (it depends on the device's SM count). Returns 0 if the
+ * parameters are invalid. The workspace must be zero-filled once before its first use (this
+ * clears the error word); afterwards the library keeps it consistent itself. One workspace must
+ * not be used by two calls that may run concurrently. */
+size_t rra_workspace_bytes(const rra_params *p);
+
+/* Step 1 (estimate). q, k: bf16 inputs. mass: fp32 output, [b, Hq, NB(NB+1)/2] packed rows
+ * summing to 1. The pooled keys and the per-row partial sums live in the workspace. */
+rra_status rra_estimate(const rra_params *p, const void *q, const void *k, float *mass,
+                        void *workspace, size_t workspace_bytes, rra_stream_t stream);
+
+/* Step 2 (select). mass: fp32 [b, Hq, NB(NB+1)/2] (any non-negative values; negative or NaN
+ * entries count as 0). For each row: sort J descending by mass (ties: smaller J first), keep the
+ * shortest prefix whose running sum, accumulated in fp64, reaches tau * (fp64 row sum), add the
+ * diagonal J = I, emit ascending. tau >= 1 keeps every block. Outputs kept_idx, kept_cnt. */
+rra_status rra_select(const rra_params *p, const float *mass, int32_t *kept_idx,
+                      int32_t *kept_cnt, rra_stream_t stream);
+
+/* Step 3 (attention). out[b, h, t, :] = softmax over the keys u of the kept blocks of t's block
+ * row with u <= t of (softmax_scale * q_t . k_u), applied to v; bf16 output, fp32 accumulation.
+ * Any kept list is accepted (it need not contain the diagonal); a query with no key gets 0.
+ * List entries that are out of [0, I] or not strictly ascending are skipped and flag
+ * RRA_ERR_INVALID_ARG in the workspace error word. */
+rra_status rra_sparse_attn(const rra_params *p, const void *q, const void *k, const void *v,
+                           const int32_t *kept_idx, const int32_t *kept_cnt, void *out,
+                           void *workspace, size_t workspace_bytes, rra_stream_t stream);
+
+/* Steps 1-3 back to back on one stream. mass may be NULL (then it lives in the workspace,
+ * which rra_workspace_bytes accounts for). kept_idx / kept_cnt are outputs. */
+rra_status rra_prefill(const rra_params *p, const void *q, const void *k, const void *v,
+                       void *out, float *mass, int32_t *kept_idx, int32_t *kept_cnt,
+                       void *workspace, size_t workspace_bytes, rra_stream_t stream);
+
+/* Synchronises `stream`, reads the workspace error word and clears it. Returns RRA_OK,
+ * RRA_ERR_DEVICE_TIMEOUT (a barrier wait expired), RRA_ERR_INVALID_ARG (a kept list was
+ * invalid) or RRA_ERR_CUDA. If raw_word is non-NULL the raw word is stored there. */
+rra_status rra_check_device_status(void *workspace, rra_stream_t stream, uint32_t *raw_word);
+
+/* Static description of a status code. */
+const char *rra_status_string(rra_status s);
+
+/* Library version, e.g. "rra 0.1 sm_100a". */
+const char *rra_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RRA_H_ */

@@ -1,0 +1,482 @@
+// Round-robin block-importance estimation (RRAttention, abstract and "Summary": one query per
+// stride per head at an offset that rotates across heads, stride-pooled keys, stride-level
+// softmax, block aggregation).
+//
+//   K1 pool_keys_kernel   Kbar[kv, j] = sum_{t<S} K[kv, j*S + t]  (fp32 sum, stored as bf16 hi+lo)
+//   K2 rr_estimate_kernel z[h, i, j] = scale * Q[h, i*S + o_h] . Kbar[kv(h), j] on tcgen05,
+//                         causal (j <= i) stride softmax, block masses
+//                         A[h, I, J] = (1/m) sum_{i in I} sum_{j in J} P[h, i, j].
+//
+// K2 is a persistent, warp-specialised kernel. One work item is (batch, head, tile of 128
+// sampled queries); the CTA streams the 128-stride key tiles n = 0..t through a 2-stage TMA
+// ring, the MMA warp computes each 128x128 logit tile into one of two TMEM accumulators as
+// Qhat . Kbar_hi + Qhat . Kbar_lo (bf16 operands, fp32 accumulation, ~16-bit Kbar), and eight
+// epilogue warps (two per TMEM lane quadrant, one per 64-column half) take the online causal
+// softmax. Because a row's normaliser is known only after its last tile, each thread writes its
+// per-(row, key block) partial sums with the running maximum they were taken against into a
+// per-CTA scratch slot (L2-resident), then rescales them once the row is complete and reduces
+// the m sampled rows of each block row with warp shuffles.
+#include <math.h>
+
+#include "common.cuh"
+#include "rra_internal.h"
+
+namespace rra {
+
+// ---------------------------------------------------------------------------------- K1
+template <int S>
+__global__ void __launch_bounds__(256) pool_keys_kernel(const uint4 *__restrict__ k,
+                                                        uint4 *__restrict__ khi,
+                                                        uint4 *__restrict__ klo,
+                                                        int64_t out_rows, int vec_per_row) {
+  const int64_t total = out_rows * vec_per_row;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = idx / vec_per_row;
+    const int v = static_cast<int>(idx - row * vec_per_row);
+    const uint4 *src = k + (row * S) * vec_per_row + v;
+    uint4 x[S];
+#pragma unroll
+    for (int t = 0; t < S; ++t) x[t] = __ldg(src + static_cast<int64_t>(t) * vec_per_row);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int t = 0; t < S; ++t) {
+      const __nv_bfloat162 *p = reinterpret_cast<const __nv_bfloat162 *>(&x[t]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(p[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+    uint4 hi, lo;
+    uint32_t *ph = reinterpret_cast<uint32_t *>(&hi);
+    uint32_t *pl = reinterpret_cast<uint32_t *>(&lo);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(acc[2 * e], acc[2 * e + 1]);
+      const float2 hf = __bfloat1622float2(h2);
+      const __nv_bfloat162 l2 = __floats2bfloat162_rn(acc[2 * e] - hf.x, acc[2 * e + 1] - hf.y);
+      ph[e] = *reinterpret_cast<const uint32_t *>(&h2);
+      pl[e] = *reinterpret_cast<const uint32_t *>(&l2);
+    }
+    khi[idx] = hi;
+    klo[idx] = lo;
+  }
+}
+
+// ---------------------------------------------------------------------------------- K2
+struct EstParams {
+  int hq, hkv, g, ns, ntiles, shift, S;
+  int n_items;       // b * hq * ntiles
+  int bhq;           // b * hq
+  float scale_log2;  // softmax scale * log2(e)
+  int64_t tri;       // packed entries per (batch, head)
+  float *mass;
+  float *est_e;
+  float *est_ref;
+  uint32_t *status;
+};
+
+// Work items in longest-first order: the first b*hq items are the last query tile of every
+// head (t = ntiles-1, the most key tiles), then t = ntiles-2, and so on.
+__device__ __forceinline__ void est_decode(const EstParams &p, int item, int &bh, int &t) {
+  const int level = item / p.bhq;
+  bh = item - level * p.bhq;
+  t = p.ntiles - 1 - level;
+}
+
+template <int D, int M>
+__global__ void __launch_bounds__(384, 1)
+    rr_estimate_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_khi,
+                       const __grid_constant__ CUtensorMap tm_klo, const EstParams p) {
+  constexpr int NCHUNK = D / 64;                  // 64-column (128-byte) chunks per row
+  constexpr uint32_t CHUNK_BYTES = 128 * 128;     // 128 rows x 128 bytes
+  constexpr uint32_t TILE_BYTES = NCHUNK * CHUNK_BYTES;
+  constexpr int NSTAGE = 2;
+  constexpr int SEG = 64 / M;                     // key blocks per 64-column half tile
+  constexpr int SEG_ROW = 128 / M;                // key blocks per 128-stride key tile
+  constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sQ = smem;
+  uint8_t *sK = smem + TILE_BYTES;                // stage s: hi at s*2*TILE, lo at +TILE
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sK + NSTAGE * 2 * TILE_BYTES);
+  uint64_t *q_full = bars + 0;
+  uint64_t *q_empty = bars + 1;
+  uint64_t *kv_full = bars + 2;                   // [NSTAGE]
+  uint64_t *kv_empty = bars + 4;                  // [NSTAGE]
+  uint64_t *acc_full = bars + 6;                  // [2]
+  uint64_t *acc_empty = bars + 8;                 // [2]
+  uint64_t *drain = bars + 10;
+  float *sM = reinterpret_cast<float *>(bars + 12);   // [2][128]
+  float *sL = sM + 256;                               // [2][128]
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sL + 256);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (grid_timed_out(p.status)) return;   // uniform across the CTA
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 256);
+    }
+    mbar_init(drain, 1);
+    *s_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(s_tmem, 256);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_khi);
+    tma_prefetch_desc(&tm_klo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, qph = 0;
+      int issued_q = 0;
+      int issued[NSTAGE] = {0, 0};
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        int bh, t;
+        est_decode(p, item, bh, t);
+        const int h = bh % p.hq;
+        const int b = bh / p.hq;
+        const int kv = h / p.g;
+        const int o = ((h + p.shift) % p.S + p.S) % p.S;
+        if (issued_q > 0) {
+          if (!mbar_wait(q_empty, qph, s_abort, p.status)) break;
+          qph ^= 1;
+        }
+        mbar_arrive_expect_tx(q_full, TILE_BYTES);
+        for (int c = 0; c < NCHUNK; ++c)
+          tma_load_3d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, o, bh * p.ns + t * 128);
+        ++issued_q;
+        const int krow = (b * p.hkv + kv) * p.ns;
+        for (int n = 0; n <= t; ++n) {
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&kv_full[stage], 2 * TILE_BYTES);
+          uint8_t *hi = sK + stage * 2 * TILE_BYTES;
+          for (int c = 0; c < NCHUNK; ++c) {
+            tma_load_2d(hi + c * CHUNK_BYTES, &tm_khi, &kv_full[stage], c * 64, krow + n * 128);
+            tma_load_2d(hi + TILE_BYTES + c * CHUNK_BYTES, &tm_klo, &kv_full[stage], c * 64,
+                        krow + n * 128);
+          }
+          ++issued[stage];
+          if (++stage == NSTAGE) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*s_abort) {   // let every copy already issued land before the CTA exits
+        if (issued_q > 0) mbar_wait_drain(q_full, (issued_q - 1) & 1);
+        for (int s = 0; s < NSTAGE; ++s)
+          if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, qph = 0, aph = 0;
+      int acc = 0;
+      bool ok = true;
+      const uint32_t q_base = smem_u32(sQ);
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        int bh, t;
+        est_decode(p, item, bh, t);
+        if (!mbar_wait(q_full, qph, s_abort, p.status)) break;
+        qph ^= 1;
+        for (int n = 0; n <= t; ++n) {
+          if (!mbar_wait(&acc_empty[acc], aph ^ 1, s_abort, p.status) ||
+              !mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + acc * 128;
+          const uint32_t k_base = smem_u32(sK + stage * 2 * TILE_BYTES);
+#pragma unroll
+          for (int part = 0; part < 2; ++part)
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t a = sdesc_kmajor_sw128(q_base + c * CHUNK_BYTES + kk * 32);
+                const uint64_t bd = sdesc_kmajor_sw128(k_base + part * TILE_BYTES +
+                                                       c * CHUNK_BYTES + kk * 32);
+                mma_bf16_ss(d_tmem, a, bd, IDESC, (part | c | kk) != 0);
+              }
+          mma_commit(&kv_empty[stage]);
+          mma_commit(&acc_full[acc]);
+          if (++stage == NSTAGE) {
+            stage = 0;
+            phase ^= 1;
+          }
+          if (++acc == 2) {
+            acc = 0;
+            aph ^= 1;
+          }
+        }
+        if (ok) mma_commit(q_empty);
+      }
+      mma_commit(drain);   // every MMA issued by this thread completes before teardown
+      mbar_wait_drain(drain, 0);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax / mass epilogue
+    const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
+    const int half = (warp - 4) >> 2;     // accumulator columns 64*half .. 64*half+63
+    const int r = quad * 32 + lane;       // row of the 128-row query tile
+    const float NEG_INF = -INFINITY;
+    int acc = 0;
+    uint32_t aph = 0;
+    bool dead = false;
+    float *e_base = p.est_e + static_cast<size_t>(blockIdx.x * 128 + r) * p.ntiles * SEG_ROW;
+    float *ref_base = p.est_ref + static_cast<size_t>(blockIdx.x * 128 + r) * p.ntiles * 2;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+      int bh, t;
+      est_decode(p, item, bh, t);
+      const int i = t * 128 + r;          // sampled query (stride) index of this row
+      const bool row_ok = i < p.ns;
+      float m_run = NEG_INF, l_run = 0.f;
+      for (int n = 0; n <= t; ++n) {
+        if (!dead) dead = !mbar_wait_warp(&acc_full[acc], aph, s_abort, p.status);
+        float e[SEG];
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) e[s] = 0.f;
+        if (!dead) {
+          tc_fence_after();
+          uint32_t u[64];
+          const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * 128 +
+                                 half * 64;
+          tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&acc_empty[acc]);
+          if (row_ok) {
+            const int j0 = n * 128 + half * 64;
+            float x[64];
+            float tmax = NEG_INF;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+              const float v = __uint_as_float(u[c]) * p.scale_log2;
+              x[c] = (j0 + c <= i) ? v : NEG_INF;
+              tmax = fmaxf(tmax, x[c]);
+            }
+            if (tmax > m_run) {
+              l_run *= fast_exp2(m_run - tmax);    // m_run = -inf: exp2(-inf) = 0
+              m_run = tmax;
+            }
+            if (m_run > NEG_INF) {
+#pragma unroll
+              for (int s = 0; s < SEG; ++s) {
+                float acc_s = 0.f;
+#pragma unroll
+                for (int c = 0; c < M; ++c) acc_s += fast_exp2(x[s * M + c] - m_run);
+                e[s] = acc_s;
+                l_run += acc_s;
+              }
+            }
+          }
+        }
+        if (++acc == 2) {
+          acc = 0;
+          aph ^= 1;
+        }
+        float *dst = e_base + static_cast<size_t>(n) * SEG_ROW + half * SEG;
+        if constexpr (SEG % 4 == 0) {
+#pragma unroll
+          for (int s = 0; s < SEG; s += 4)
+            *reinterpret_cast<float4 *>(dst + s) = make_float4(e[s], e[s + 1], e[s + 2], e[s + 3]);
+        } else {
+#pragma unroll
+          for (int s = 0; s < SEG; s += 2)
+            *reinterpret_cast<float2 *>(dst + s) = make_float2(e[s], e[s + 1]);
+        }
+        ref_base[n * 2 + half] = m_run;
+      }
+      // ---- combine the two half-rows' running max / sum
+      sM[half * 128 + r] = m_run;
+      sL[half * 128 + r] = l_run;
+      named_bar_sync(1, 256);
+      const float m0 = sM[r], m1 = sM[128 + r];
+      const float mx = fmaxf(m0, m1);
+      float ltot = 0.f;
+      if (m0 > NEG_INF) ltot += sL[r] * fast_exp2(m0 - mx);
+      if (m1 > NEG_INF) ltot += sL[128 + r] * fast_exp2(m1 - mx);
+      named_bar_sync(1, 256);
+      const float inv = (row_ok && ltot > 0.f) ? 1.f / ltot : 0.f;
+      // ---- rescale the partial sums and reduce the M sampled rows of each block row
+      const int I = i / M;
+      float *mass_row = p.mass + static_cast<int64_t>(bh) * p.tri +
+                        static_cast<int64_t>(I) * (I + 1) / 2;
+      const bool writer = row_ok && ((lane % M) == 0);
+      for (int n = 0; n <= t; ++n) {
+        const float mref = ref_base[n * 2 + half];
+        const float f = (inv > 0.f && mref > NEG_INF) ? fast_exp2(mref - mx) * inv : 0.f;
+        const float *src = e_base + static_cast<size_t>(n) * SEG_ROW + half * SEG;
+        float e[SEG];
+        if constexpr (SEG % 4 == 0) {
+#pragma unroll
+          for (int s = 0; s < SEG; s += 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(src + s);
+            e[s] = v.x; e[s + 1] = v.y; e[s + 2] = v.z; e[s + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int s = 0; s < SEG; s += 2) {
+            const float2 v = *reinterpret_cast<const float2 *>(src + s);
+            e[s] = v.x; e[s + 1] = v.y;
+          }
+        }
+        const int jb0 = (n * 128 + half * 64) / M;
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) {
+          float v = e[s] * f;
+#pragma unroll
+          for (int off = M / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+          const int J = jb0 + s;
+          if (writer && J <= I) mass_row[J] = v * (1.f / M);
+        }
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---------------------------------------------------------------------------------- launch
+static bool make_map(CUtensorMap *map, void *base, int rank, const cuuint64_t *dims,
+                     const cuuint64_t *strides_bytes, const cuuint32_t *box) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return false;
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides_bytes, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+cudaError_t launch_pool_keys(const Geometry &g, const void *k, void *khi, void *klo,
+                             int num_sms, cudaStream_t stream) {
+  const int64_t out_rows = static_cast<int64_t>(g.b) * g.hkv * g.ns;
+  const int vec = g.d / 8;
+  const int64_t total = out_rows * vec;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const uint4 *src = static_cast<const uint4 *>(k);
+  uint4 *hi = static_cast<uint4 *>(khi), *lo = static_cast<uint4 *>(klo);
+  switch (g.S) {
+    case 4: pool_keys_kernel<4><<<blocks, threads, 0, stream>>>(src, hi, lo, out_rows, vec); break;
+    case 8: pool_keys_kernel<8><<<blocks, threads, 0, stream>>>(src, hi, lo, out_rows, vec); break;
+    case 16: pool_keys_kernel<16><<<blocks, threads, 0, stream>>>(src, hi, lo, out_rows, vec); break;
+    case 32: pool_keys_kernel<32><<<blocks, threads, 0, stream>>>(src, hi, lo, out_rows, vec); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <int D, int M>
+static cudaError_t launch_est_t(const CUtensorMap &mq, const CUtensorMap &mhi,
+                                const CUtensorMap &mlo, const EstParams &ep, int slots,
+                                cudaStream_t stream) {
+  constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
+  const size_t smem = 1024 + TILE * (1 + 2 * 2) + 12 * 8 + 512 * 4 + 16;
+  auto kern = rr_estimate_kernel<D, M>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<slots, 384, smem, stream>>>(mq, mhi, mlo, ep);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rr_estimate(const Geometry &g, const void *q, const void *khi,
+                               const void *klo, float *mass, float *est_e, float *est_ref,
+                               int slots, uint32_t *status, cudaStream_t stream) {
+  CUtensorMap mq, mhi, mlo;
+  const cuuint64_t bhq_ns = static_cast<cuuint64_t>(g.b) * g.hq * g.ns;
+  const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.S), bhq_ns};
+  const cuuint64_t qstr[2] = {static_cast<cuuint64_t>(g.d) * 2,
+                              static_cast<cuuint64_t>(g.S) * g.d * 2};
+  const cuuint32_t qbox[3] = {64, 1, 128};
+  if (!make_map(&mq, const_cast<void *>(q), 3, qdims, qstr, qbox)) return cudaErrorInvalidValue;
+  const cuuint64_t kdims[2] = {static_cast<cuuint64_t>(g.d),
+                               static_cast<cuuint64_t>(g.b) * g.hkv * g.ns};
+  const cuuint64_t kstr[1] = {static_cast<cuuint64_t>(g.d) * 2};
+  const cuuint32_t kbox[2] = {64, 128};
+  if (!make_map(&mhi, const_cast<void *>(khi), 2, kdims, kstr, kbox)) return cudaErrorInvalidValue;
+  if (!make_map(&mlo, const_cast<void *>(klo), 2, kdims, kstr, kbox)) return cudaErrorInvalidValue;
+
+  EstParams ep;
+  ep.hq = g.hq;
+  ep.hkv = g.hkv;
+  ep.g = g.g;
+  ep.ns = g.ns;
+  ep.ntiles = g.ntiles;
+  ep.shift = g.shift;
+  ep.S = g.S;
+  ep.bhq = g.b * g.hq;
+  ep.n_items = ep.bhq * g.ntiles;
+  ep.scale_log2 = g.scale * 1.4426950408889634f;
+  ep.tri = g.tri;
+  ep.mass = mass;
+  ep.est_e = est_e;
+  ep.est_ref = est_ref;
+  ep.status = status;
+  if (slots > ep.n_items) slots = ep.n_items;
+  if (g.d == 128) {
+    switch (g.m) {
+      case 4: return launch_est_t<128, 4>(mq, mhi, mlo, ep, slots, stream);
+      case 8: return launch_est_t<128, 8>(mq, mhi, mlo, ep, slots, stream);
+      case 16: return launch_est_t<128, 16>(mq, mhi, mlo, ep, slots, stream);
+      case 32: return launch_est_t<128, 32>(mq, mhi, mlo, ep, slots, stream);
+    }
+  } else if (g.d == 64) {
+    switch (g.m) {
+      case 4: return launch_est_t<64, 4>(mq, mhi, mlo, ep, slots, stream);
+      case 8: return launch_est_t<64, 8>(mq, mhi, mlo, ep, slots, stream);
+      case 16: return launch_est_t<64, 16>(mq, mhi, mlo, ep, slots, stream);
+      case 32: return launch_est_t<64, 32>(mq, mhi, mlo, ep, slots, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace rra

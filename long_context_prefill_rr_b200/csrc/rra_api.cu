@@ -1,0 +1,243 @@
+// C ABI of the RRAttention prefill hot path (declared in include/rra.h): argument validation,
+// workspace carve-up and kernel launches. No memory is allocated here.
+#include <math.h>
+#include <mutex>
+
+#include "../../include/rra.h"
+#include "common.cuh"
+#include "rra_internal.h"
+
+namespace rra {
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+WorkspaceLayout workspace_layout(const Geometry &g, int num_sms) {
+  WorkspaceLayout w{};
+  size_t off = 256;   // header: status word
+  w.status = 0;
+  const size_t kbar = static_cast<size_t>(g.b) * g.hkv * g.ns * g.d * 2;
+  w.khi = align_up(off, 1024);
+  off = w.khi + kbar;
+  w.klo = align_up(off, 1024);
+  off = w.klo + kbar;
+  const int64_t items = static_cast<int64_t>(g.b) * g.hq * g.ntiles;
+  int slots = num_sms < 1 ? 1 : num_sms;
+  if (items < slots) slots = static_cast<int>(items < 1 ? 1 : items);
+  w.est_slots = slots;
+  const int segs = g.m > 0 ? 128 / g.m : 0;
+  w.est_e = align_up(off, 256);
+  off = w.est_e + static_cast<size_t>(slots) * 128 * g.ntiles * segs * 4;
+  w.est_ref = align_up(off, 256);
+  off = w.est_ref + static_cast<size_t>(slots) * 128 * g.ntiles * 2 * 4;
+  w.mass = align_up(off, 256);
+  off = w.mass + static_cast<size_t>(g.b) * g.hq * g.tri * 4;
+  w.total = align_up(off, 256);
+  return w;
+}
+
+EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+}  // namespace rra
+
+using rra::Geometry;
+using rra::WorkspaceLayout;
+
+namespace {
+
+enum Needs : unsigned { kNeedsStride = 1u, kNeedsHeadDim = 2u };
+
+// Checks the shape parameters and resolves the geometry. `needs` says which kernel limits apply
+// (the estimate needs a supported stride, the estimate and the attention a supported head_dim).
+rra_status resolve(const rra_params *p, unsigned needs, Geometry *g) {
+  if (!p) return RRA_ERR_INVALID_ARG;
+  if (p->batch < 0 || p->seqlen < 0 || p->heads_q < 1 || p->heads_kv < 1 ||
+      p->heads_q % p->heads_kv != 0 || p->block <= 0 || p->stride <= 0 || p->head_dim <= 0)
+    return RRA_ERR_INVALID_ARG;
+  if (p->seqlen % p->block != 0 || p->block % p->stride != 0) return RRA_ERR_INVALID_ARG;
+  if (!(p->tau > 0.f)) return RRA_ERR_INVALID_ARG;   // also rejects NaN
+  if (p->block != 128) return RRA_ERR_UNSUPPORTED;
+  if ((needs & kNeedsHeadDim) && p->head_dim != 64 && p->head_dim != 128)
+    return RRA_ERR_UNSUPPORTED;
+  if ((needs & kNeedsStride) && p->stride != 4 && p->stride != 8 && p->stride != 16 &&
+      p->stride != 32)
+    return RRA_ERR_UNSUPPORTED;
+  // TMA coordinates and row indices are 32-bit
+  const int64_t rows_q = static_cast<int64_t>(p->batch) * p->heads_q * p->seqlen;
+  if (rows_q >= (static_cast<int64_t>(1) << 31)) return RRA_ERR_UNSUPPORTED;
+  g->b = p->batch;
+  g->hq = p->heads_q;
+  g->hkv = p->heads_kv;
+  g->L = p->seqlen;
+  g->d = p->head_dim;
+  g->B = p->block;
+  g->S = p->stride;
+  g->shift = ((p->shift % p->stride) + p->stride) % p->stride;
+  g->g = p->heads_q / p->heads_kv;
+  g->m = p->block / p->stride;
+  g->nb = p->seqlen / p->block;
+  g->ns = p->seqlen / p->stride;
+  g->ntiles = (g->ns + 127) / 128;
+  g->tri = static_cast<int64_t>(g->nb) * (g->nb + 1) / 2;
+  g->tau = p->tau;
+  g->scale = p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / sqrtf(static_cast<float>(p->head_dim));
+  return RRA_OK;
+}
+
+bool empty(const Geometry &g) { return g.b == 0 || g.L == 0; }
+
+bool ptr_ok(const void *ptr) {
+  return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+  return n;
+}
+
+rra_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RRA_OK : RRA_ERR_CUDA; }
+
+uint32_t *status_word(void *ws, const WorkspaceLayout &w) {
+  return reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + w.status);
+}
+
+template <class T>
+T *ws_at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
+}
+
+rra_status run_estimate(const Geometry &g, const void *q, const void *k, float *mass, void *ws,
+                        const WorkspaceLayout &w, int sms, cudaStream_t st) {
+  cudaError_t e = rra::launch_pool_keys(g, k, ws_at<void>(ws, w.khi), ws_at<void>(ws, w.klo),
+                                        sms, st);
+  if (e != cudaSuccess) return RRA_ERR_CUDA;
+  e = rra::launch_rr_estimate(g, q, ws_at<void>(ws, w.khi), ws_at<void>(ws, w.klo), mass,
+                              ws_at<float>(ws, w.est_e), ws_at<float>(ws, w.est_ref),
+                              w.est_slots, status_word(ws, w), st);
+  return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t rra_workspace_bytes(const rra_params *p) {
+  Geometry g;
+  if (resolve(p, 0, &g) != RRA_OK) return 0;
+  const int sms = num_sms();
+  if (sms <= 0) return 0;
+  return rra::workspace_layout(g, sms).total;
+}
+
+rra_status rra_estimate(const rra_params *p, const void *q, const void *k, float *mass,
+                        void *workspace, size_t workspace_bytes, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, kNeedsStride | kNeedsHeadDim, &g);
+  if (s != RRA_OK) return s;
+  if (empty(g)) return RRA_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(mass) || !ptr_ok(workspace)) return RRA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return RRA_ERR_CUDA;
+  const WorkspaceLayout w = rra::workspace_layout(g, sms);
+  if (workspace_bytes < w.total) return RRA_ERR_WORKSPACE;
+  return run_estimate(g, q, k, mass, workspace, w, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rra_status rra_select(const rra_params *p, const float *mass, int32_t *kept_idx,
+                      int32_t *kept_cnt, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, 0, &g);
+  if (s != RRA_OK) return s;
+  if (empty(g)) return RRA_OK;
+  if (!ptr_ok(mass) || !ptr_ok(kept_idx) || !ptr_ok(kept_cnt)) return RRA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return RRA_ERR_CUDA;
+  return cuda_status(rra::launch_topt_select(g, mass, kept_idx, kept_cnt, sms,
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rra_status rra_sparse_attn(const rra_params *p, const void *q, const void *k, const void *v,
+                           const int32_t *kept_idx, const int32_t *kept_cnt, void *out,
+                           void *workspace, size_t workspace_bytes, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, kNeedsHeadDim, &g);
+  if (s != RRA_OK) return s;
+  if (empty(g)) return RRA_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(kept_idx) || !ptr_ok(kept_cnt) ||
+      !ptr_ok(out) || !ptr_ok(workspace))
+    return RRA_ERR_INVALID_ARG;
+  if (workspace_bytes < 256) return RRA_ERR_WORKSPACE;   // only the status word is used
+  return cuda_status(rra::launch_sparse_attn(g, q, k, v, kept_idx, kept_cnt, out,
+                                             static_cast<uint32_t *>(workspace),
+                                             reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rra_status rra_prefill(const rra_params *p, const void *q, const void *k, const void *v,
+                       void *out, float *mass, int32_t *kept_idx, int32_t *kept_cnt,
+                       void *workspace, size_t workspace_bytes, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, kNeedsStride | kNeedsHeadDim, &g);
+  if (s != RRA_OK) return s;
+  if (empty(g)) return RRA_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(out) || !ptr_ok(kept_idx) ||
+      !ptr_ok(kept_cnt) || !ptr_ok(workspace) || (mass != nullptr && !ptr_ok(mass)))
+    return RRA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return RRA_ERR_CUDA;
+  const WorkspaceLayout w = rra::workspace_layout(g, sms);
+  if (workspace_bytes < w.total) return RRA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  float *m = mass ? mass : ws_at<float>(workspace, w.mass);
+  s = run_estimate(g, q, k, m, workspace, w, sms, st);
+  if (s != RRA_OK) return s;
+  if (rra::launch_topt_select(g, m, kept_idx, kept_cnt, sms, st) != cudaSuccess)
+    return RRA_ERR_CUDA;
+  return cuda_status(rra::launch_sparse_attn(g, q, k, v, kept_idx, kept_cnt, out,
+                                             status_word(workspace, w), st));
+}
+
+rra_status rra_check_device_status(void *workspace, rra_stream_t stream, uint32_t *raw_word) {
+  if (!ptr_ok(workspace)) return RRA_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return RRA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RRA_ERR_CUDA;
+  if (raw_word) *raw_word = word;
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return RRA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return RRA_ERR_CUDA;
+  }
+  if (word & rra::kErrTimeout) return RRA_ERR_DEVICE_TIMEOUT;
+  if (word & rra::kErrBadList) return RRA_ERR_INVALID_ARG;
+  return RRA_OK;
+}
+
+const char *rra_status_string(rra_status s) {
+  switch (s) {
+    case RRA_OK: return "ok";
+    case RRA_ERR_INVALID_ARG: return "invalid argument";
+    case RRA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RRA_ERR_WORKSPACE: return "workspace too small";
+    case RRA_ERR_CUDA: return "CUDA error";
+    case RRA_ERR_DEVICE_TIMEOUT: return "device barrier wait timed out";
+  }
+  return "unknown status";
+}
+
+const char *rra_version(void) { return "rra 0.1 sm_100a"; }
+
+}  // extern "C"

@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on seeded inputs.
+
+Small workloads are compared element by element (every mass, every kept list, every output
+row); the long-context workloads at their full sizes are compared on seeded samples of block
+rows, which the oracle computes one by one, plus the exact agreement of the GPU's select with
+the oracle's select run on the GPU's own masses over every row.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as orc
+import parity as par
+from long_context_prefill_rr_b200 import native
+from long_context_prefill_rr_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _prepare(w):
+    qb, kb, vb = wl.make_workload(w)
+    return (qb, kb, vb), (par.to_dev(qb), par.to_dev(kb), par.to_dev(vb))
+
+
+def _full_check(w, p, bits, gpu, label):
+    qb, kb, vb = bits
+    q64, k64, v64 = (wl.bf16_bits_to_f64(x) for x in bits)
+    scale = par.resolved_scale(p)
+    nb = w.seqlen // w.block
+    assert gpu["status"] == 0, f"{label}: device status {gpu['raw']:#x}"
+    om = orc.estimate(q64, k64, w.block, w.stride, w.shift, scale)
+    merr = float(np.abs(gpu["mass"] - om).max())
+    assert merr <= par.MASS_ATOL, f"{label}: mass err {merr}"
+    assert par.select_on_gpu_masses_exact(gpu, w.tau, nb), f"{label}: select on GPU masses"
+    rows = {(b, h, I): om[b, h, orc.tri_offset(I):orc.tri_offset(I + 1)]
+            for b in range(w.batch) for h in range(w.heads_q) for I in range(nb)}
+    mism, exc, n = par.compare_select_rows(gpu, rows, w.tau)
+    assert not mism, f"{label}: kept-list mismatches outside the boundary rule: {mism[:5]}"
+    ref = orc.sparse_attention(q64, k64, v64, gpu["idx"], gpu["cnt"], w.block, scale)
+    ma, rr = par.attention_errors(gpu["out"], ref)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, f"{label}: attn {ma} {rr}"
+    dens = gpu["cnt"].sum() / (w.batch * w.heads_q * orc.tri_offset(nb))
+    print(f"[{label}] mass_err={merr:.3g} boundary_rows={len(exc)}/{n} attn_max={ma:.3g} "
+          f"attn_rrms={rr:.3g} density={dens:.3f}")
+
+
+def test_tiny_full_parity(cuda_device):
+    w, p = par.workload_params(wl.WORKLOADS["tiny"])
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    _full_check(w, p, bits, gpu, "tiny")
+
+
+@pytest.mark.parametrize("label,over", [
+    ("s4_shift3_tau0.8", dict(stride=4, shift=3, tau=0.8)),
+    ("s16_shiftm1_scale", dict(stride=16, shift=-1, tau=0.95, softmax_scale=0.125)),
+    ("s32_default_scale", dict(stride=32, shift=5, tau=0.5, softmax_scale=-1.0)),
+    ("gqa4_d128_ragged", dict(heads_q=8, heads_kv=2, head_dim=128, seqlen=1152, stride=8)),
+    ("batch2_short", dict(batch=2, seqlen=768, stride=16, heads_q=4, heads_kv=4)),
+    ("one_block", dict(seqlen=128, stride=8)),
+])
+def test_tiny_variants_full_parity(cuda_device, label, over):
+    w, p = par.workload_params(wl.WORKLOADS["tiny"], **over)
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    _full_check(w, p, bits, gpu, label)
+
+
+def test_tau_one_is_dense_causal(cuda_device):
+    """tau = 1 keeps every causal block and the output is dense causal attention."""
+    w, p = par.workload_params(wl.WORKLOADS["tiny"], tau=1.0, heads_q=8, heads_kv=2,
+                               head_dim=128)
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    nb = w.seqlen // w.block
+    assert (gpu["cnt"] == np.arange(1, nb + 1)[None, None, :]).all()
+    q64, k64, v64 = (wl.bf16_bits_to_f64(x) for x in bits)
+    qt = torch.from_numpy(q64)
+    kt = torch.from_numpy(k64).repeat_interleave(4, dim=1)
+    vt = torch.from_numpy(v64).repeat_interleave(4, dim=1)
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True,
+                                                           scale=1.0).numpy()
+    ma, rr = par.attention_errors(gpu["out"], ref)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (ma, rr)
+
+
+@pytest.mark.parametrize("density,d", [(0.5, 128), (0.15, 128), (0.3, 64)])
+def test_sparse_attn_random_masks(cuda_device, density, d):
+    """rra_sparse_attn on caller-supplied random masks, including a row without its diagonal
+    and an empty row, against the oracle."""
+    w, p = par.workload_params(wl.WORKLOADS["tiny"], heads_q=8, heads_kv=2, head_dim=d,
+                               seqlen=2048)
+    bits, dev = _prepare(w)
+    nb = w.seqlen // w.block
+    idx, cnt = wl.random_kept_lists(1, 8, nb, density, seed=11)
+    off = orc.tri_offset(5)
+    idx[0, 3, off:off + 6] = [0, 2, -1, -1, -1, -1]   # no diagonal
+    cnt[0, 3, 5] = 2
+    off = orc.tri_offset(9)
+    idx[0, 6, off:off + 10] = -1                      # empty row
+    cnt[0, 6, 9] = 0
+    out = torch.empty_like(dev[0])
+    ws = native.new_workspace(p)
+    native.sparse_attn(p, *dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), out,
+                       ws)
+    st, raw = native.check_device_status(ws)
+    assert st == 0, raw
+    q64, k64, v64 = (wl.bf16_bits_to_f64(x) for x in bits)
+    ref = orc.sparse_attention(q64, k64, v64, idx, cnt, w.block, 1.0)
+    ma, rr = par.attention_errors(par.bf16_dev_to_f32(out), ref)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (ma, rr)
+    o = par.bf16_dev_to_f32(out)
+    assert (o[0, 6, 9 * 128:10 * 128] == 0).all()
+
+
+def test_invalid_list_entries_are_skipped_and_flagged(cuda_device):
+    w, p = par.workload_params(wl.WORKLOADS["tiny"], heads_q=2, heads_kv=2)
+    bits, dev = _prepare(w)
+    nb = w.seqlen // w.block
+    idx, cnt = wl.random_kept_lists(1, 2, nb, 1.0, seed=3)
+    off = orc.tri_offset(4)
+    idx[0, 1, off:off + 5] = [1, 0, 3, 9, 4]   # 0 not ascending, 9 > I: both skipped
+    cnt[0, 1, 4] = 5
+    out = torch.empty_like(dev[0])
+    ws = native.new_workspace(p)
+    native.sparse_attn(p, *dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), out,
+                       ws)
+    st, raw = native.check_device_status(ws)
+    assert st == 1 and raw == 2
+    st2, raw2 = native.check_device_status(ws)
+    assert st2 == 0 and raw2 == 0                   # cleared by the first read
+    idx[0, 1, off:off + 5] = [1, 3, 4, -1, -1]      # the valid subsequence
+    cnt[0, 1, 4] = 3
+    q64, k64, v64 = (wl.bf16_bits_to_f64(x) for x in bits)
+    ref = orc.sparse_attention(q64, k64, v64, idx, cnt, w.block, 1.0)
+    ma, rr = par.attention_errors(par.bf16_dev_to_f32(out), ref)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (ma, rr)
+
+
+def test_select_edge_cases(cuda_device):
+    """All-zero rows, exact ties, a single dominant block and tau = 1, on rra_select alone,
+    against the oracle's select on the same fp32 masses."""
+    p = native.params(1, 4, 4, 1024, 64, 8, 0.9)
+    nb = 8
+    T = orc.tri_offset(nb)
+    rng = np.random.default_rng(5)
+    m = rng.random((1, 4, T)).astype(np.float32)
+    m[0, 0] = 0.0                                            # head 0: all zero
+    m[0, 1] = 0.25                                           # head 1: all tied
+    m[0, 2] = 1e-6
+    for I in range(nb):
+        m[0, 2, orc.tri_offset(I)] = 1.0                     # head 2: dominant J = 0
+    for tau in (0.9, 0.5, 1.0):
+        p.tau = tau
+        md = torch.from_numpy(m).cuda()
+        idx = torch.empty((1, 4, T), dtype=torch.int32, device="cuda")
+        cnt = torch.empty((1, 4, nb), dtype=torch.int32, device="cuda")
+        native.select(p, md, idx, cnt)
+        ri, rc = orc.select(m.astype(np.float64), nb, float(np.float32(tau)))
+        assert np.array_equal(idx.cpu().numpy(), ri) and np.array_equal(cnt.cpu().numpy(), rc)
+
+
+def test_empty_problem(cuda_device):
+    p = native.params(0, 8, 8, 1024, 64, 8, 0.9)
+    z = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    assert native.load().rra_prefill(native._p(p), *([native._ptr(z)] * 8), 16,
+                                     native._stream(None)) == 0
+
+
+def _sampled_check(w, p, bits, gpu, label, n_rows, n_attn_rows, seed):
+    qb, kb, vb = bits
+    assert gpu["status"] == 0, f"{label}: device status {gpu['raw']:#x}"
+    nb = w.seqlen // w.block
+    assert par.select_on_gpu_masses_exact(gpu, w.tau, nb), f"{label}: select on GPU masses"
+    qc, kc, vc = par.HeadCache(qb), par.HeadCache(kb), par.HeadCache(vb)
+    rows = par.sample_rows(p, n_rows, seed)
+    om = par.oracle_mass_rows(qc, kc, p, rows)
+    merr = max(float(np.abs(gpu["mass"][b, h, orc.tri_offset(I):orc.tri_offset(I + 1)] -
+                            om[(b, h, I)]).max()) for b, h, I in rows)
+    assert merr <= par.MASS_ATOL, f"{label}: mass err {merr}"
+    mism, exc, n = par.compare_select_rows(gpu, om, w.tau)
+    assert not mism, f"{label}: kept-list mismatches: {mism[:5]}"
+    arows = rows[:n_attn_rows] + [rows[-1]] if n_attn_rows < len(rows) else rows
+    arows = sorted(set(arows))
+    ref = par.oracle_attention_rows(qc, kc, vc, p, gpu["idx"], gpu["cnt"], arows)
+    ma, rr = par.attention_rows_errors(gpu["out"], ref)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, f"{label}: attn {ma} {rr}"
+    dens = gpu["cnt"].sum(dtype=np.int64) / (w.batch * w.heads_q * orc.tri_offset(nb))
+    print(f"[{label}] mass_err={merr:.3g} boundary_rows={len(exc)}/{n} attn_max={ma:.3g} "
+          f"attn_rrms={rr:.3g} density={dens:.4f}")
+
+
+def test_llama8k_parity(cuda_device):
+    w, p = par.workload_params(wl.WORKLOADS["llama8k"])
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    _sampled_check(w, p, bits, gpu, "llama8k", n_rows=256, n_attn_rows=48, seed=1)
+
+
+@pytest.mark.parametrize("S,tau", [(8, 0.9), (16, 0.95)])
+def test_llama32k_parity(cuda_device, S, tau):
+    w, p = par.workload_params(wl.WORKLOADS["llama32k"], stride=S, tau=tau)
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    _sampled_check(w, p, bits, gpu, f"llama32k_S{S}_tau{tau}", n_rows=64, n_attn_rows=16, seed=2)
+
+
+def test_video64k_parity(cuda_device):
+    w, p = par.workload_params(wl.WORKLOADS["video64k"])
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    _sampled_check(w, p, bits, gpu, "video64k", n_rows=64, n_attn_rows=16, seed=4)
+
+
+def test_llama128k_parity(cuda_device):
+    w, p = par.workload_params(wl.WORKLOADS["llama128k"])
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    del dev
+    torch.cuda.empty_cache()
+    _sampled_check(w, p, bits, gpu, "llama128k", n_rows=48, n_attn_rows=12, seed=3)
