@@ -268,10 +268,13 @@ __global__ void __launch_bounds__(256, 1)
       }
       if (j == 0) {
         m_run = tmax;
-      } else if (tmax > m_run + RESCALE_THRESHOLD) {
-        const float alpha = fast_exp2(m_run - tmax);
+      } else if (__any_sync(0xffffffffu, tmax > m_run + RESCALE_THRESHOLD)) {
+        // Warp-uniform: the TMEM accesses below are warp-collective. Lanes whose own max did
+        // not move get alpha = 1.
+        const float m_new = fmaxf(m_run, tmax);
+        const float alpha = fast_exp2(m_run - m_new);
         l_run *= alpha;
-        m_run = tmax;
+        m_run = m_new;
         // O must be final for tile j-1 before it is rescaled (the PV of tile j waits for us).
         if (!mbar_wait_warp(o_done, (j - 1) & 1, s_abort, p.status)) {
           dead = true;
