@@ -182,6 +182,17 @@ def _dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings over the process group (identity when there is
+    none); every rank takes this collective at the same point."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.cpu()]
+
+
 def run_reference(args, w):
     ws, rank, _ = _dist_env()
     if rank != 0:
@@ -294,10 +305,7 @@ def run_gpu(args, w):
     torch.cuda.synchronize(dev)
     e2e_ms = e_start.elapsed_time(e_stop) / e_steps
 
-    t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-    if ws_n > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     if rank == 0:
         peaks = _peaks()

@@ -6,6 +6,10 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+# tests/test_oracle_mutations.py runs the oracle pins against a mutated copy of the oracle
+_ORACLE_OVERRIDE = os.environ.get("RRA_ORACLE_OVERRIDE")
+if _ORACLE_OVERRIDE:
+    sys.path.insert(0, _ORACLE_OVERRIDE)
 
 
 def pytest_configure(config):
