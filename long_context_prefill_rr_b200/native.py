@@ -32,6 +32,8 @@ _SIGS = {
     "rra_prefill": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                _c.c_void_p]),
+    "rra_estimate_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                               _c.c_void_p, _c.c_void_p]),
     "rra_check_device_status": (_c.c_int, [_c.c_void_p, _c.c_void_p,
                                            _c.POINTER(_c.c_uint32)]),
     "rra_status_string": (_c.c_char_p, [_c.c_int]),
@@ -144,6 +146,19 @@ def estimate(p: RraParams, q, k, mass, ws, stream=None):
     _expect(mass, torch.float32, sh["mass"], "mass")
     _check(load().rra_estimate(_p(p), _ptr(q), _ptr(k), _ptr(mass), _ptr(ws), ws.numel(),
                                _stream(stream)), "rra_estimate")
+
+
+def estimate_static_scratch(p: RraParams, q, k, mass, stream=None):
+    """rra_estimate without a workspace, for callers that cannot allocate device memory: the
+    library's fixed 32 MiB device array serves as scratch (problems that need more are
+    refused; calls that overlap on the GPU race on the shared array)."""
+    import torch
+    sh = shapes(p)
+    _expect(q, torch.bfloat16, sh["q"], "q")
+    _expect(k, torch.bfloat16, sh["kv"], "k")
+    _expect(mass, torch.float32, sh["mass"], "mass")
+    _check(load().rra_estimate_static_scratch(_p(p), _ptr(q), _ptr(k), _ptr(mass),
+                                              _stream(stream)), "rra_estimate_static_scratch")
 
 
 def select(p: RraParams, mass, kept_idx, kept_cnt, stream=None):
