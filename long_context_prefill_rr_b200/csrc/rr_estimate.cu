@@ -284,28 +284,42 @@ __global__ void __launch_bounds__(384, 1)
           tc_fence_before();
           mbar_arrive(&acc_empty[acc]);
           if (row_ok) {
-            const int j0 = n * 128 + half * 64;
-            float x[64];
-            float tmax = NEG_INF;
+            float *uf = reinterpret_cast<float *>(u);
+            if (n == t) {   // diagonal key tile: stride j is visible to sampled query i iff j <= i
+              const int j0 = n * 128 + half * 64;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-              const float v = __uint_as_float(u[c]) * p.scale_log2;
-              x[c] = (j0 + c <= i) ? v : NEG_INF;
-              tmax = fmaxf(tmax, x[c]);
+              for (int c = 0; c < 64; ++c)
+                if (j0 + c > i) uf[c] = -INFINITY;
             }
+            float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+#pragma unroll
+            for (int c = 0; c < 64; c += 8) {
+              mx[0] = fmax3(mx[0], uf[c], uf[c + 1]);
+              mx[1] = fmax3(mx[1], uf[c + 2], uf[c + 3]);
+              mx[2] = fmax3(mx[2], uf[c + 4], uf[c + 5]);
+              mx[3] = fmax3(mx[3], uf[c + 6], uf[c + 7]);
+            }
+            const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * p.scale_log2;
             if (tmax > m_run) {
               l_run *= fast_exp2(m_run - tmax);    // m_run = -inf: exp2(-inf) = 0
               m_run = tmax;
             }
             if (m_run > NEG_INF) {
+              const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+              const uint64_t negm = f2_pack(-m_run, -m_run);
+              uint64_t tot = 0;
 #pragma unroll
               for (int s = 0; s < SEG; ++s) {
-                float acc_s = 0.f;
+                uint64_t acc2 = 0;
 #pragma unroll
-                for (int c = 0; c < M; ++c) acc_s += fast_exp2(x[s * M + c] - m_run);
-                e[s] = acc_s;
-                l_run += acc_s;
+                for (int c = 0; c < M; c += 2) {
+                  const uint64_t xy = ffma2(f2_pack(uf[s * M + c], uf[s * M + c + 1]), sl2, negm);
+                  acc2 = fadd2(acc2, f2_pack(fast_exp2(f2_lo(xy)), fast_exp2(f2_hi(xy))));
+                }
+                e[s] = f2_lo(acc2) + f2_hi(acc2);
+                tot = fadd2(tot, acc2);
               }
+              l_run += f2_lo(tot) + f2_hi(tot);
             }
           }
         }

@@ -2,18 +2,23 @@
 // the selected blocks; "regular block-sparse FlashAttention execution" in the RBS-Attention
 // digest; online softmax as in FlashAttention / FlashAttention-2), GQA head mapping.
 //
-// One CTA per (batch, head, query block I), launched longest-first (I descending). Roles:
-//   warp 0      TMA producer: Q tile once, then K_0, K_1, V_0, K_2, V_1, ... through a 3-stage
-//               ring (the order the MMA warp consumes them in);
-//   warp 1      MMA issuer (one thread): S_j = Q K_j^T into TMEM buffer j%2 (tcgen05, bf16 ->
-//               fp32), then O += P_{j-1} V_{j-1} with P from shared memory, so the softmax of
-//               tile j overlaps the PV product of tile j-1 and the QK product of tile j+1;
-//   warp 2      TMEM allocation (S0 | S1 | O);
-//   warps 4-7   softmax: one thread per query row reads its 128 logits from TMEM, applies the
-//               causal mask on the diagonal block, keeps a running max (rescaling O in TMEM
-//               only when the max grows by more than 2^8) and running sum, writes P as bf16
-//               into the 128B-swizzled K-major layout the MMA reads, and finally normalises O
-//               and stores the bf16 row.
+// One CTA runs two work items side by side: query block I of heads 2c and 2c+1 (of one batch
+// row), each with its own kept list. Grid order is longest-first (I descending). Roles:
+//   warp 0       TMA producer: both Q tiles once, then per step j the tiles V_A(j-1), K_A(j),
+//                V_B(j-1), K_B(j) through a ring of 128-row tiles, in the order the MMA warp
+//                consumes them;
+//   warp 1       MMA issuer (one thread), same order: O_X += P_X V_X(j-1) with P read from TMEM
+//                (tcgen05 "TS" form), then S_X = Q_X K_X(j)^T into the same TMEM columns. While
+//                one item's softmax runs, the tensor core works on the other item (ping-pong);
+//   warp 2       TMEM allocation: S/P_A | S/P_B | O_A | O_B (512 columns for d = 128);
+//   warps 4-7    softmax of item A, warps 8-11 softmax of item B: one thread per query row reads
+//                its 128 logits from TMEM, masks the diagonal block, keeps a running max (O is
+//                rescaled in TMEM only when the max grows by more than 2^8, decided per warp)
+//                and running sum, writes P as bf16 back over S, and at the end normalises O
+//                and stores the bf16 row.
+// Because the S/P columns of an item are reused every tile, S_X(j) completing implies the
+// previous PV product of that item completed (MMAs complete in issue order), so O_X is stable
+// whenever its softmax runs.
 // The kept list is read by every role with the same validity rule (0 <= J <= I, strictly
 // ascending); invalid entries are skipped and flagged in the status word by the producer.
 #include <math.h>
@@ -24,7 +29,8 @@
 namespace rra {
 
 struct AttnParams {
-  int hq, hkv, g, L, nb, bhq;
+  int hq, hkv, g, L, nb, batch;
+  int n_pairs;       // batch * ceil(hq / 2)
   int64_t tri;
   float scale_log2;
   const int32_t *kept_idx;
@@ -33,24 +39,45 @@ struct AttnParams {
   uint32_t *status;
 };
 
-// Clamp the stored count to the row's capacity (I + 1 entries).
-__device__ __forceinline__ int row_count(const AttnParams &p, int bh, int I) {
-  int cnt = p.kept_cnt[static_cast<int64_t>(bh) * p.nb + I];
-  if (cnt < 0) cnt = 0;
-  if (cnt > I + 1) cnt = I + 1;
-  return cnt;
-}
+// Walks one kept row, yielding the valid entries (0 <= J <= I, strictly ascending).
+struct ListCursor {
+  const int32_t *lst;
+  int cnt, e, prev, I;
+  __device__ void init(const AttnParams &p, int bh, int I_, bool valid) {
+    I = I_;
+    e = 0;
+    prev = -1;
+    lst = p.kept_idx + static_cast<int64_t>(bh) * p.tri + static_cast<int64_t>(I) * (I + 1) / 2;
+    cnt = 0;
+    if (valid) {
+      cnt = p.kept_cnt[static_cast<int64_t>(bh) * p.nb + I];
+      if (cnt < 0) cnt = 0;
+      if (cnt > I + 1) cnt = I + 1;
+    }
+  }
+  // next valid block index, or -1; invalid entries are reported through `status` if non-null
+  __device__ int next(uint32_t *status) {
+    while (e < cnt) {
+      const int J = lst[e++];
+      if (J > prev && J <= I) {
+        prev = J;
+        return J;
+      }
+      if (status) atomicOr(status, kErrBadList);
+    }
+    return -1;
+  }
+};
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bs_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   constexpr int NCHUNK = D / 64;
   constexpr uint32_t CHUNK_BYTES = 128 * 128;
   constexpr uint32_t TILE_BYTES = NCHUNK * CHUNK_BYTES;   // 128 rows x D bf16
-  constexpr uint32_t P_BYTES = 2 * CHUNK_BYTES;           // 128 rows x 128 keys bf16
-  constexpr int NSTAGE = 3;
+  constexpr int NSTAGE = (D == 128) ? 5 : 10;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false);
   constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, true);
   constexpr float RESCALE_THRESHOLD = 8.0f;               // log2 units
@@ -58,32 +85,36 @@ __global__ void __launch_bounds__(256, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sQ = smem;
-  uint8_t *sRing = sQ + TILE_BYTES;
-  uint8_t *sP = sRing + NSTAGE * TILE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(sP + 2 * P_BYTES);
+  uint8_t *sQ = smem;                               // [2] tiles
+  uint8_t *sRing = sQ + 2 * TILE_BYTES;             // [NSTAGE] tiles
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sRing + NSTAGE * TILE_BYTES);
   uint64_t *q_full = bars + 0;
-  uint64_t *kv_full = bars + 1;       // [NSTAGE]
-  uint64_t *kv_empty = bars + 4;      // [NSTAGE]
-  uint64_t *s_full = bars + 7;        // [2]
-  uint64_t *p_full = bars + 9;        // [2]
-  uint64_t *o_done = bars + 11;
-  uint64_t *o_final = bars + 12;
-  uint64_t *drain = bars + 13;
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 14);
+  uint64_t *kv_full = bars + 1;                     // [NSTAGE]
+  uint64_t *kv_empty = kv_full + NSTAGE;            // [NSTAGE]
+  uint64_t *s_full = kv_empty + NSTAGE;             // [2]
+  uint64_t *p_full = s_full + 2;                    // [2]
+  uint64_t *o_final = p_full + 2;                   // [2]
+  uint64_t *drain = o_final + 2;
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int level = blockIdx.x / p.bhq;
-  const int bh = blockIdx.x - level * p.bhq;
+  const int level = blockIdx.x / p.n_pairs;
+  const int pair = blockIdx.x - level * p.n_pairs;
   const int I = p.nb - 1 - level;
-  const int h = bh % p.hq;
-  const int b = bh / p.hq;
-  const int kv = h / p.g;
-  const int32_t *lst = p.kept_idx + static_cast<int64_t>(bh) * p.tri +
-                       static_cast<int64_t>(I) * (I + 1) / 2;
-  const int cnt = row_count(p, bh, I);
+  const int hp = (p.hq + 1) >> 1;
+  const int b = pair / hp;
+  const int h0 = 2 * (pair - b * hp);
+  int bh[2], kvrow[2];
+  bool valid[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int h = h0 + x;
+    valid[x] = h < p.hq;
+    bh[x] = b * p.hq + (valid[x] ? h : h0);
+    kvrow[x] = (b * p.hkv + (valid[x] ? h : h0) / p.g) * p.L;
+  }
 
   if (grid_timed_out(p.status)) return;   // uniform across the CTA
   if (threadIdx.x == 0) {
@@ -92,12 +123,11 @@ __global__ void __launch_bounds__(256, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_final[x], 1);
     }
-    mbar_init(o_done, 1);
-    mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -115,23 +145,24 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t tmem_o = tmem + 256;
+  // columns: S/P of item x at 128*x, O of item x at 256 + D*x
+  auto tm_s = [&](int x) { return tmem + 128u * x; };
+  auto tm_o = [&](int x) { return tmem + 256u + static_cast<uint32_t>(D) * x; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      int issued[NSTAGE] = {0, 0, 0};
-      bool q_issued = false, ok = true;
-      const int qrow = bh * p.L + I * 128;
-      const int kvrow = (b * p.hkv + kv) * p.L;
-      auto load = [&](const CUtensorMap *map, int J) -> bool {
+      int issued[NSTAGE];
+      for (int s = 0; s < NSTAGE; ++s) issued[s] = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap *map, int row) -> bool {
         if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) return false;
         mbar_arrive_expect_tx(&kv_full[stage], TILE_BYTES);
         uint8_t *dst = sRing + stage * TILE_BYTES;
         for (int c = 0; c < NCHUNK; ++c)
-          tma_load_2d(dst + c * CHUNK_BYTES, map, &kv_full[stage], c * 64, kvrow + J * 128);
+          tma_load_2d(dst + c * CHUNK_BYTES, map, &kv_full[stage], c * 64, row);
         ++issued[stage];
         if (++stage == NSTAGE) {
           stage = 0;
@@ -139,28 +170,40 @@ __global__ void __launch_bounds__(256, 1)
         }
         return true;
       };
-      int prev = -1, last = -1, j = 0;
-      for (int e = 0; e < cnt && ok; ++e) {
-        const int J = lst[e];
-        if (!(J > prev && J <= I)) {
-          atomicOr(p.status, kErrBadList);
-          continue;
-        }
-        prev = J;
-        if (!q_issued) {
-          mbar_arrive_expect_tx(q_full, TILE_BYTES);
-          for (int c = 0; c < NCHUNK; ++c)
-            tma_load_2d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, qrow);
-          q_issued = true;
-        }
-        ok = load(&tm_k, J);
-        if (ok && j >= 1) ok = load(&tm_v, last);
-        last = J;
-        ++j;
+      ListCursor cur[2];
+      int J[2], pendV[2] = {-1, -1};
+      for (int x = 0; x < 2; ++x) {
+        cur[x].init(p, bh[x], I, valid[x]);
+        J[x] = cur[x].next(p.status);
       }
-      if (ok && j >= 1) ok = load(&tm_v, last);
+      const bool q_any = J[0] >= 0 || J[1] >= 0;
+      if (q_any) {
+        mbar_arrive_expect_tx(q_full, TILE_BYTES * ((J[0] >= 0) + (J[1] >= 0)));
+        for (int x = 0; x < 2; ++x)
+          if (J[x] >= 0)
+            for (int c = 0; c < NCHUNK; ++c)
+              tma_load_2d(sQ + x * TILE_BYTES + c * CHUNK_BYTES, &tm_q, q_full, c * 64,
+                          bh[x] * p.L + I * 128);
+      }
+      while (ok) {
+        bool any = false;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (pendV[x] >= 0) {
+            ok = load(&tm_v, kvrow[x] + pendV[x] * 128);
+            pendV[x] = -1;
+            any = true;
+          }
+          if (ok && J[x] >= 0) {
+            ok = load(&tm_k, kvrow[x] + J[x] * 128);
+            pendV[x] = J[x];
+            J[x] = cur[x].next(p.status);
+            any = true;
+          }
+        }
+        if (!any) break;
+      }
       if (*s_abort) {
-        if (q_issued) mbar_wait_drain(q_full, 0);
+        if (q_any) mbar_wait_drain(q_full, 0);
         for (int s = 0; s < NSTAGE; ++s)
           if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
       }
@@ -170,177 +213,211 @@ __global__ void __launch_bounds__(256, 1)
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true;
+      bool ok = true, q_ready = false;
       const uint32_t q_base = smem_u32(sQ);
-      const uint32_t p_base = smem_u32(sP);
-      auto issue_pv = [&](int jj) -> bool {
-        if (!mbar_wait(&p_full[jj & 1], (jj >> 1) & 1, s_abort, p.status)) return false;
-        if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(sRing + stage * TILE_BYTES);
-        const uint32_t pb = p_base + (jj & 1) * P_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t a = sdesc_kmajor_sw128(pb + (kk >> 2) * CHUNK_BYTES + (kk & 3) * 32);
-          const uint64_t bd = sdesc_mnmajor_sw128(v_base + kk * 2048, CHUNK_BYTES);
-          mma_bf16_ss(tmem_o, a, bd, IDESC_O, (jj > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&kv_empty[stage]);
-        mma_commit(o_done);
-        if (++stage == NSTAGE) {
-          stage = 0;
-          phase ^= 1;
-        }
-        return true;
-      };
-      int prev = -1, j = 0;
-      for (int e = 0; e < cnt && ok; ++e) {
-        const int J = lst[e];
-        if (!(J > prev && J <= I)) continue;
-        prev = J;
-        if (j == 0 && !mbar_wait(q_full, 0, s_abort, p.status)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(sRing + stage * TILE_BYTES);
-        const uint32_t s_tm = tmem + (j & 1) * 128;
-#pragma unroll
-        for (int c = 0; c < NCHUNK; ++c)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t a = sdesc_kmajor_sw128(q_base + c * CHUNK_BYTES + kk * 32);
-            const uint64_t bd = sdesc_kmajor_sw128(k_base + c * CHUNK_BYTES + kk * 32);
-            mma_bf16_ss(s_tm, a, bd, IDESC_S, (c | kk) != 0);
-          }
-        mma_commit(&kv_empty[stage]);
-        mma_commit(&s_full[j & 1]);
-        if (++stage == NSTAGE) {
-          stage = 0;
-          phase ^= 1;
-        }
-        if (j >= 1) ok = issue_pv(j - 1);
-        ++j;
+      ListCursor cur[2];
+      int J[2], ntile[2] = {0, 0};
+      bool pend[2] = {false, false};
+      for (int x = 0; x < 2; ++x) {
+        cur[x].init(p, bh[x], I, valid[x]);
+        J[x] = cur[x].next(nullptr);
       }
-      if (ok && j >= 1) {
-        ok = issue_pv(j - 1);
-        if (ok) mma_commit(o_final);
+      while (ok) {
+        bool any = false;
+        for (int x = 0; x < 2 && ok; ++x) {
+          if (pend[x]) {
+            // O_x += P_x(t) V_x(t), t = ntile[x] - 1; P sits in the S columns of item x
+            const int t = ntile[x] - 1;
+            if (!mbar_wait(&p_full[x], t & 1, s_abort, p.status) ||
+                !mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t v_base = smem_u32(sRing + stage * TILE_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const uint64_t bd = sdesc_mnmajor_sw128(v_base + kk * 2048, CHUNK_BYTES);
+              mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, bd, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+            }
+            mma_commit(&kv_empty[stage]);
+            if (J[x] < 0) mma_commit(&o_final[x]);
+            if (++stage == NSTAGE) {
+              stage = 0;
+              phase ^= 1;
+            }
+            pend[x] = false;
+            any = true;
+          }
+          if (J[x] >= 0) {
+            if (!q_ready) {
+              if (!mbar_wait(q_full, 0, s_abort, p.status)) {
+                ok = false;
+                break;
+              }
+              q_ready = true;
+            }
+            if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_base = smem_u32(sRing + stage * TILE_BYTES);
+            const uint32_t qx = q_base + x * TILE_BYTES;
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t a = sdesc_kmajor_sw128(qx + c * CHUNK_BYTES + kk * 32);
+                const uint64_t bd = sdesc_kmajor_sw128(k_base + c * CHUNK_BYTES + kk * 32);
+                mma_bf16_ss(tm_s(x), a, bd, IDESC_S, (c | kk) != 0);
+              }
+            mma_commit(&kv_empty[stage]);
+            mma_commit(&s_full[x]);
+            if (++stage == NSTAGE) {
+              stage = 0;
+              phase ^= 1;
+            }
+            ++ntile[x];
+            pend[x] = true;
+            J[x] = cur[x].next(nullptr);
+            any = true;
+          }
+        }
+        if (!any) break;
       }
       mma_commit(drain);
       mbar_wait_drain(drain, 0);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
+    const int x = (warp - 4) >> 2;       // item
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t s_cols = tm_s(x) + lane_off;
+    const uint32_t o_cols = tm_o(x) + lane_off;
     const float NEG_INF = -INFINITY;
-    float m_run = NEG_INF, l_run = 0.f;
-    int prev = -1, j = 0;
+    const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    float m_run = NEG_INF;
+    uint64_t lsum[4] = {0, 0, 0, 0};
     bool dead = false;
-    for (int e = 0; e < cnt && !dead; ++e) {
-      const int J = lst[e];
-      if (!(J > prev && J <= I)) continue;
-      prev = J;
-      if (!mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1, s_abort, p.status)) {
+    ListCursor cur;
+    cur.init(p, bh[x], I, valid[x]);
+    int t = 0;
+    for (int J = cur.next(nullptr); J >= 0; J = cur.next(nullptr), ++t) {
+      if (!mbar_wait_warp(&s_full[x], t & 1, s_abort, p.status)) {
         dead = true;
         break;
       }
       tc_fence_after();
-      float x[128];
+      const bool diag = (J == I);   // diagonal block: key c is visible to query r iff c <= r
+      // pass 1: row max over the 128 logits, 64 columns at a time
+      float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float u[64];
+        tmem_ld32(s_cols + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(s_cols + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_ld_wait();
+        if (diag) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem + lane_off + (j & 1) * 128 + c * 32,
-                  *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
-      tmem_ld_wait();
-      const bool diag = (J == I);
-      float tmax = NEG_INF;
+          for (int c = 0; c < 64; ++c)
+            if (h * 64 + c > r) u[c] = NEG_INF;
+        }
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = x[c] * p.scale_log2;
-        if (diag && c > r) v = NEG_INF;
-        x[c] = v;
-        tmax = fmaxf(tmax, v);
+        for (int c = 0; c < 64; c += 8) {
+          mx[0] = fmax3(mx[0], u[c], u[c + 1]);
+          mx[1] = fmax3(mx[1], u[c + 2], u[c + 3]);
+          mx[2] = fmax3(mx[2], u[c + 4], u[c + 5]);
+          mx[3] = fmax3(mx[3], u[c + 6], u[c + 7]);
+        }
       }
-      if (j == 0) {
+      const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * sl2;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (t == 0) {
         m_run = tmax;
       } else if (__any_sync(0xffffffffu, tmax > m_run + RESCALE_THRESHOLD)) {
-        // Warp-uniform: the TMEM accesses below are warp-collective. Lanes whose own max did
-        // not move get alpha = 1.
         const float m_new = fmaxf(m_run, tmax);
-        const float alpha = fast_exp2(m_run - m_new);
-        l_run *= alpha;
+        alpha = fast_exp2(m_run - m_new);
         m_run = m_new;
-        // O must be final for tile j-1 before it is rescaled (the PV of tile j waits for us).
-        if (!mbar_wait_warp(o_done, (j - 1) & 1, s_abort, p.status)) {
-          dead = true;
-          break;
+        rescale = true;
+        // the sum so far was taken against the old max; this tile's terms are added below
+        const uint64_t a2 = f2_pack(alpha, alpha);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) lsum[c] = fmul2(lsum[c], a2);
+      }
+      // pass 2: P = 2^(u*scale_log2 - m) in bf16, written over S. Keys 0..63 are re-read and
+      // packed into columns 0..31 before keys 64..127 are re-read: the packed P of keys 64..127
+      // lands in columns 32..63, whose logits (keys 32..63) are consumed by then.
+      const uint64_t negm = f2_pack(-m_run, -m_run);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        float u[64];
+        tmem_ld32(s_cols + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(s_cols + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_ld_wait();
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (h * 64 + c > r) u[c] = NEG_INF;
         }
-        tc_fence_after();
+        uint32_t pk[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const uint64_t xy = ffma2(f2_pack(u[2 * q], u[2 * q + 1]), sl2x2, negm);
+          const float p0 = fast_exp2(f2_lo(xy));
+          const float p1 = fast_exp2(f2_hi(xy));
+          lsum[q & 3] = fadd2(lsum[q & 3], f2_pack(p0, p1));
+          pk[q] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(s_cols + h * 32, pk);
+      }
+      if (rescale) {
+        // O_x is final for the previous tile: S_x(t) completing implies it
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld32(o_cols + c * 32, o);
           tmem_ld_wait();
 #pragma unroll
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(tmem_o + lane_off + c * 32, o);
-        }
-        tmem_st_wait();
-      }
-      // P = 2^(x - m) as bf16 into the swizzled K-major tile (two 64-key chunks)
-      uint8_t *prow = sP + (j & 1) * P_BYTES + r * 128;
-      float lsum = 0.f;
-#pragma unroll
-      for (int kc = 0; kc < 2; ++kc) {
-#pragma unroll
-        for (int piece = 0; piece < 8; ++piece) {
-          uint32_t w[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int c = kc * 64 + piece * 8 + q * 2;
-            const float p0 = fast_exp2(x[c] - m_run);
-            const float p1 = fast_exp2(x[c + 1] - m_run);
-            lsum += p0 + p1;
-            w[q] = pack_bf16x2(p0, p1);
-          }
-          *reinterpret_cast<uint4 *>(prow + kc * CHUNK_BYTES + ((piece ^ (r & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          tmem_st32(o_cols + c * 32, o);
         }
       }
-      l_run += lsum;
-      fence_proxy_async_smem();
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[j & 1]);
-      ++j;
+      mbar_arrive(&p_full[x]);
     }
-    __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh) * p.L + I * 128 + r) * D;
-    if (!dead && j > 0 && mbar_wait_warp(o_final, 0, s_abort, p.status)) {
-      tc_fence_after();
-      const float inv = 1.f / l_run;
+    if (valid[x]) {
+      __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh[x]) * p.L + I * 128 + r) * D;
+      if (!dead && t > 0 && mbar_wait_warp(&o_final[x], 0, s_abort, p.status)) {
+        tc_fence_after();
+        const uint64_t s01 = fadd2(lsum[0], lsum[1]), s23 = fadd2(lsum[2], lsum[3]);
+        const uint64_t s4 = fadd2(s01, s23);
+        const float inv = 1.f / (f2_lo(s4) + f2_hi(s4));
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tmem_o + lane_off + c * 32, o);
-        tmem_ld_wait();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_cols + c * 32, o);
+          tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 32; q += 8) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[q]) * inv, __uint_as_float(o[q + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv);
-          *reinterpret_cast<uint4 *>(orow + c * 32 + q) = v;
+          for (int q = 0; q < 32; q += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[q]) * inv, __uint_as_float(o[q + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv);
+            *reinterpret_cast<uint4 *>(orow + c * 32 + q) = v;
+          }
         }
-      }
-    } else if (j == 0) {
+      } else if (!dead && t == 0) {
 #pragma unroll
-      for (int c = 0; c < D; c += 8)
-        *reinterpret_cast<uint4 *>(orow + c) = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < D; c += 8)
+          *reinterpret_cast<uint4 *>(orow + c) = make_uint4(0, 0, 0, 0);
+      }
     }
     tc_fence_before();
   }
@@ -356,12 +433,13 @@ static cudaError_t launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk,
                                  const CUtensorMap &mv, const AttnParams &ap, int64_t grid,
                                  cudaStream_t stream) {
   constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
-  const size_t smem = 1024 + TILE * (1 + 3) + 2 * 2 * 128 * 128 + 14 * 8 + 16;
+  constexpr int NSTAGE = (D == 128) ? 5 : 10;
+  const size_t smem = 1024 + TILE * (2 + NSTAGE) + (1 + 2 * NSTAGE + 7) * 8 + 16;
   auto kern = bs_attn_fwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(grid), 256, smem, stream>>>(mq, mk, mv, ap);
+  kern<<<static_cast<unsigned>(grid), 384, smem, stream>>>(mq, mk, mv, ap);
   return cudaGetLastError();
 }
 
@@ -392,14 +470,15 @@ cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, 
   ap.g = g.g;
   ap.L = g.L;
   ap.nb = g.nb;
-  ap.bhq = g.b * g.hq;
+  ap.batch = g.b;
+  ap.n_pairs = g.b * ((g.hq + 1) / 2);
   ap.tri = g.tri;
   ap.scale_log2 = g.scale * 1.4426950408889634f;
   ap.kept_idx = kept_idx;
   ap.kept_cnt = kept_cnt;
   ap.out = static_cast<__nv_bfloat16 *>(out);
   ap.status = status;
-  const int64_t grid = static_cast<int64_t>(ap.bhq) * g.nb;
+  const int64_t grid = static_cast<int64_t>(ap.n_pairs) * g.nb;
   if (g.d == 128) return launch_attn_t<128>(mq, mk, mv, ap, grid, stream);
   if (g.d == 64) return launch_attn_t<64>(mq, mk, mv, ap, grid, stream);
   return cudaErrorInvalidValue;

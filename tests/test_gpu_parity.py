@@ -84,6 +84,35 @@ def test_tau_one_is_dense_causal(cuda_device):
     assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (ma, rr)
 
 
+def test_attention_rescale_divergent_rows(cuda_device):
+    """Rows whose running max jumps by far more than the lazy-rescale threshold in a later
+    block (only every other query row, so the rescale decision differs across a warp) still
+    match the oracle."""
+    w, p = par.workload_params(wl.WORKLOADS["tiny"], heads_q=4, heads_kv=2, head_dim=128,
+                               seqlen=1024)
+    qb, kb, vb = wl.make_workload(w)
+    q = wl.bf16_bits_to_f32(qb)
+    k = wl.bf16_bits_to_f32(kb)
+    u = np.zeros(w.head_dim, np.float32)
+    u[7] = 1.0
+    q[:, :, ::2, :] += 4.0 * u                  # even query rows lean along u
+    k[:, :, 3 * 128:4 * 128, :] += 5.0 * u      # keys of block 3 point along u: +20 logit jump
+    qb, kb = wl.bf16_round_bits(q), wl.bf16_round_bits(k)
+    nb = w.seqlen // w.block
+    idx, cnt = wl.random_kept_lists(1, 4, nb, 1.0, seed=0)
+    dev = [par.to_dev(x) for x in (qb, kb, vb)]
+    out = torch.empty_like(dev[0])
+    ws = native.new_workspace(p)
+    native.sparse_attn(p, *dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), out,
+                       ws)
+    st, raw = native.check_device_status(ws)
+    assert st == 0, raw
+    q64, k64, v64 = (wl.bf16_bits_to_f64(x) for x in (qb, kb, vb))
+    ref = orc.sparse_attention(q64, k64, v64, idx, cnt, w.block, 1.0)
+    ma, rr = par.attention_errors(par.bf16_dev_to_f32(out), ref)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (ma, rr)
+
+
 @pytest.mark.parametrize("density,d", [(0.5, 128), (0.15, 128), (0.3, 64)])
 def test_sparse_attn_random_masks(cuda_device, density, d):
     """rra_sparse_attn on caller-supplied random masks, including a row without its diagonal
@@ -219,32 +248,3 @@ def test_llama128k_parity(cuda_device):
     del dev
     torch.cuda.empty_cache()
     _sampled_check(w, p, bits, gpu, "llama128k", n_rows=48, n_attn_rows=12, seed=3)
-
-
-def test_attention_rescale_divergent_rows(cuda_device):
-    """Rows whose running max jumps by far more than the lazy-rescale threshold in a later
-    block (only every other query row, so the rescale decision differs across a warp) still
-    match the oracle."""
-    w, p = par.workload_params(wl.WORKLOADS["tiny"], heads_q=4, heads_kv=2, head_dim=128,
-                               seqlen=1024)
-    qb, kb, vb = wl.make_workload(w)
-    q = wl.bf16_bits_to_f32(qb)
-    k = wl.bf16_bits_to_f32(kb)
-    u = np.zeros(w.head_dim, np.float32)
-    u[7] = 1.0
-    q[:, :, ::2, :] += 4.0 * u                  # even query rows lean along u
-    k[:, :, 3 * 128:4 * 128, :] += 5.0 * u      # keys of block 3 point along u: +20 logit jump
-    qb, kb = wl.bf16_round_bits(q), wl.bf16_round_bits(k)
-    nb = w.seqlen // w.block
-    idx, cnt = wl.random_kept_lists(1, 4, nb, 1.0, seed=0)
-    dev = [par.to_dev(x) for x in (qb, kb, vb)]
-    out = torch.empty_like(dev[0])
-    ws = native.new_workspace(p)
-    native.sparse_attn(p, *dev, torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), out,
-                       ws)
-    st, raw = native.check_device_status(ws)
-    assert st == 0, raw
-    q64, k64, v64 = (wl.bf16_bits_to_f64(x) for x in (qb, kb, vb))
-    ref = orc.sparse_attention(q64, k64, v64, idx, cnt, w.block, 1.0)
-    ma, rr = par.attention_errors(par.bf16_dev_to_f32(out), ref)
-    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (ma, rr)
