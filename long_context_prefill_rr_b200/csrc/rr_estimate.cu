@@ -355,32 +355,49 @@ __global__ void __launch_bounds__(384, 1)
       float *mass_row = p.mass + static_cast<int64_t>(bh) * p.tri +
                         static_cast<int64_t>(I) * (I + 1) / 2;
       const bool writer = row_ok && ((lane % M) == 0);
-      for (int n = 0; n <= t; ++n) {
-        const float mref = ref_base[n * 2 + half];
-        const float f = (inv > 0.f && mref > NEG_INF) ? fast_exp2(mref - mx) * inv : 0.f;
-        const float *src = e_base + static_cast<size_t>(n) * SEG_ROW + half * SEG;
-        float e[SEG];
-        if constexpr (SEG % 4 == 0) {
+      // PF key tiles per batch: all their loads are issued before any is used, so the loop
+      // pays one L2 round trip per batch instead of one per tile
+      constexpr int PF = (SEG >= 32) ? 1 : 32 / SEG;
+      for (int n0 = 0; n0 <= t; n0 += PF) {
+        float fr[PF];
+        float e[PF][SEG];
 #pragma unroll
-          for (int s = 0; s < SEG; s += 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(src + s);
-            e[s] = v.x; e[s + 1] = v.y; e[s + 2] = v.z; e[s + 3] = v.w;
-          }
-        } else {
+        for (int k = 0; k < PF; ++k) {
+          const int n = n0 + k;
+          fr[k] = NEG_INF;
 #pragma unroll
-          for (int s = 0; s < SEG; s += 2) {
-            const float2 v = *reinterpret_cast<const float2 *>(src + s);
-            e[s] = v.x; e[s + 1] = v.y;
+          for (int s = 0; s < SEG; ++s) e[k][s] = 0.f;
+          if (n <= t) {
+            fr[k] = ref_base[n * 2 + half];
+            const float *src = e_base + static_cast<size_t>(n) * SEG_ROW + half * SEG;
+            if constexpr (SEG % 4 == 0) {
+#pragma unroll
+              for (int s = 0; s < SEG; s += 4) {
+                const float4 v = *reinterpret_cast<const float4 *>(src + s);
+                e[k][s] = v.x; e[k][s + 1] = v.y; e[k][s + 2] = v.z; e[k][s + 3] = v.w;
+              }
+            } else {
+#pragma unroll
+              for (int s = 0; s < SEG; s += 2) {
+                const float2 v = *reinterpret_cast<const float2 *>(src + s);
+                e[k][s] = v.x; e[k][s + 1] = v.y;
+              }
+            }
           }
         }
-        const int jb0 = (n * 128 + half * 64) / M;
 #pragma unroll
-        for (int s = 0; s < SEG; ++s) {
-          float v = e[s] * f;
+        for (int k = 0; k < PF; ++k) {
+          const int n = n0 + k;
+          const float f = (inv > 0.f && fr[k] > NEG_INF) ? fast_exp2(fr[k] - mx) * inv : 0.f;
+          const int jb0 = (n * 128 + half * 64) / M;
 #pragma unroll
-          for (int off = M / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-          const int J = jb0 + s;
-          if (writer && J <= I) mass_row[J] = v * (1.f / M);
+          for (int s = 0; s < SEG; ++s) {
+            float v = e[k][s] * f;
+#pragma unroll
+            for (int off = M / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            const int J = jb0 + s;
+            if (writer && J <= I) mass_row[J] = v * (1.f / M);
+          }
         }
       }
     }

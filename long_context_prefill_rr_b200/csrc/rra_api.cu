@@ -3,7 +3,7 @@
 #include <math.h>
 #include <mutex>
 
-#include "../../include/rra.h"
+#include "rra.h"
 #include "common.cuh"
 #include "rra_internal.h"
 

@@ -19,7 +19,7 @@
 //     capture begins.
 #include <mutex>
 
-#include "../../include/rra.h"
+#include "rra.h"
 #include "common.cuh"
 #include "rra_internal.h"
 
