@@ -332,7 +332,7 @@ def run_gpu(args, w):
             cpu = cpu_oracle_sample(w, q_bits, k_bits, v_bits, n_rows=args.ref_rows,
                                     total_kept=n_kept)
         traffic = None
-        tpath = os.path.join(ROOT, "profiles", "attn_traffic.json")
+        tpath = os.path.join(ROOT, "profiles", "bs_attn_fwd_llama128k_traffic.json")
         if os.path.exists(tpath):
             td = json.load(open(tpath))
             if td.get("workload") == w.name and td.get("kernel_rev") == KERNEL_REV:
@@ -371,7 +371,7 @@ def run_gpu(args, w):
 
 
 # bump when the attention kernel changes, so stale ncu traffic is not reported
-KERNEL_REV = "attn-v1"
+KERNEL_REV = "attn-v2"
 
 
 def main(argv=None):
