@@ -370,6 +370,83 @@ def run_gpu(args, w):
     return 0
 
 
+def run_speedup_study(args):
+    """Dense-vs-sparse study: per length, the full RR path (estimate + select + sparse
+    attention), the same attention kernel on every causal block (tau = 1: dense causal), and
+    torch's fused scaled_dot_product_attention (causal, GQA) on the same bf16 inputs, as a
+    library reference point. Prints one JSON line per length."""
+    import torch
+
+    from long_context_prefill_rr_b200 import native
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    native.load()
+    out_lines = []
+    for L in [int(x) for x in args.lengths.split(",")]:
+        w = wl.WORKLOADS["llama128k"].with_(seqlen=L, name=f"llama{L // 1024}k")
+        q_bits, k_bits, v_bits = wl.make_workload(w)
+        to = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+        q, k, v = to(q_bits), to(k_bits), to(v_bits)
+        res = {"seq_len": L}
+        for tau, name in ((w.tau, "rr"), (1.0, "dense_tau1")):
+            p = native.params(w.batch, w.heads_q, w.heads_kv, L, w.head_dim, w.stride, tau,
+                              shift=w.shift, softmax_scale=w.softmax_scale)
+            run = native.RRAttentionPrefill(p, dev)
+            out = torch.empty_like(q)
+            for _ in range(3):
+                run(q, k, v, out)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(3, min(20, int(2e9 / L / L * 4096)))
+            e0.record()
+            for _ in range(n):
+                run(q, k, v, out)
+            e1.record()
+            torch.cuda.synchronize()
+            run.check()
+            res[f"{name}_ms"] = e0.elapsed_time(e1) / n
+            if name == "rr":
+                cnt = run.kept_cnt.cpu().numpy()
+                nb = L // 128
+                res["density"] = float(cnt.sum() / (w.heads_q * nb * (nb + 1) / 2))
+            del run, out
+        g = w.heads_q // w.heads_kv
+        def sdpa():
+            return torch.nn.functional.scaled_dot_product_attention(
+                q, k, v, is_causal=True, scale=w.softmax_scale, enable_gqa=True)
+        try:
+            for _ in range(3):
+                sdpa()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            n = max(3, min(20, int(2e9 / L / L * 4096)))
+            e0.record()
+            for _ in range(n):
+                sdpa()
+            e1.record()
+            torch.cuda.synchronize()
+            res["torch_sdpa_causal_ms"] = e0.elapsed_time(e1) / n
+        except (RuntimeError, torch.cuda.OutOfMemoryError) as err:   # no fused backend: report
+            res["torch_sdpa_causal_ms"] = None
+            res["torch_sdpa_error"] = str(err).splitlines()[0][:200]
+            torch.cuda.empty_cache()
+        res["speedup_rr_vs_dense_tau1"] = res["dense_tau1_ms"] / res["rr_ms"]
+        if res["torch_sdpa_causal_ms"]:
+            res["speedup_rr_vs_torch_sdpa"] = res["torch_sdpa_causal_ms"] / res["rr_ms"]
+        dense_flops = 4.0 * w.head_dim * w.heads_q * (128 * 128 * (L // 128) * (L // 128 - 1) / 2
+                                                      + 128 * 129 / 2 * (L // 128))
+        res["dense_tau1_tflops"] = dense_flops / (res["dense_tau1_ms"] * 1e-3) / 1e12
+        if res["torch_sdpa_causal_ms"]:
+            res["torch_sdpa_tflops"] = dense_flops / (res["torch_sdpa_causal_ms"] * 1e-3) / 1e12
+        del g
+        print(json.dumps({"study": "speedup", "workload": w.name, **res}), flush=True)
+        out_lines.append(res)
+        del q, k, v
+        torch.cuda.empty_cache()
+    return 0
+
+
 # bump when the attention kernel changes, so stale ncu traffic is not reported
 KERNEL_REV = "attn-v2"
 
@@ -383,7 +460,12 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--study", choices=["speedup"], default=None,
+                    help="instead of the bench line: dense-vs-sparse speedup over --lengths")
+    ap.add_argument("--lengths", default="8192,16384,32768,65536,131072")
     args = ap.parse_args(argv)
+    if args.study == "speedup":
+        return run_speedup_study(args)
     w = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
