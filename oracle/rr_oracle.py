@@ -37,6 +37,15 @@ written at the step (and collected in the design notes of the repository):
                  scale * Q[h,t].K[kv(h),u], applied to V; a query with no key gets 0.
                  GQA: kv(h) = floor(h / (Hq/Hkv)).
 
+The XAttention antidiagonal estimator (the predecessor method, [XA] sections 2-3) replaces
+steps 1-4: within every S x S sub-block of the attention logits the S elements of the
+antidiagonal (bottom-left to top-right: query offset t with key offset S-1-t) are summed,
+
+   z^xa_{h,i,j} = scale * sum_{t<S} Q[h, i*S + t] . K[kv(h), j*S + S-1-t],  j <= i,
+
+followed by the same stride-level causal softmax, block masses (step 6) and selection (step 7).
+There is no per-head rotation: every head scores all of its queries.
+
 Parity pins for every step live in ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
@@ -46,7 +55,8 @@ import numpy as np
 __all__ = [
     "rr_offset", "pooled_keys", "block_row_logits", "stride_softmax_rows", "block_masses_row",
     "estimate", "estimate_block_row", "select_row", "select", "attention_block",
-    "sparse_attention", "tri_offset", "kv_head",
+    "sparse_attention", "tri_offset", "kv_head", "xattn_block_row_logits",
+    "xattn_estimate_block_row", "xattn_estimate",
 ]
 
 
@@ -137,6 +147,47 @@ def estimate(q: np.ndarray, k: np.ndarray, block: int, stride: int, shift: int,
             for I in range(nb):
                 out[bi, h, tri_offset(I):tri_offset(I + 1)] = estimate_block_row(
                     qh, kb, h, I, block, stride, shift, scale)
+    return out
+
+
+def xattn_block_row_logits(q: np.ndarray, k: np.ndarray, I: int, block: int, stride: int,
+                           scale: float) -> np.ndarray:
+    """Antidiagonal stride scores of block row I for one head ([XA] sections 2-3).
+
+    q [L, d] (this head's queries), k [L, d] (its KV head's keys). Returns z [m, (I+1)*m]:
+    rows i = I*m .. I*m+m-1, columns j = 0 .. (I+1)*m - 1 (j > i is masked later).
+    """
+    m = block // stride
+    L, d = q.shape
+    qs = q.astype(np.float64).reshape(L // stride, stride, d)[I * m:(I + 1) * m]   # [m, S, d]
+    ks = k.astype(np.float64).reshape(L // stride, stride, d)[:(I + 1) * m]       # [n, S, d]
+    z = np.zeros((m, (I + 1) * m))
+    for t in range(stride):
+        z += qs[:, t, :] @ ks[:, stride - 1 - t, :].T     # query offset t with key offset S-1-t
+    return scale * z
+
+
+def xattn_estimate_block_row(q: np.ndarray, k: np.ndarray, I: int, block: int, stride: int,
+                             scale: float) -> np.ndarray:
+    """XAttention masses A^xa_{h,I,0..I}: antidiagonal scores, stride softmax, block sums."""
+    m = block // stride
+    z = xattn_block_row_logits(q, k, I, block, stride, scale)
+    p = stride_softmax_rows(z, I * m)
+    return block_masses_row(p, m)
+
+
+def xattn_estimate(q: np.ndarray, k: np.ndarray, block: int, stride: int,
+                   scale: float) -> np.ndarray:
+    """All XAttention block masses, in the packed layout of ``estimate``."""
+    b, hq, hkv, L, d = _check_shapes(q, k, block, stride)
+    nb = L // block
+    out = np.zeros((b, hq, tri_offset(nb)), dtype=np.float64)
+    for bi in range(b):
+        for h in range(hq):
+            kh = k[bi, kv_head(h, hq, hkv)]
+            for I in range(nb):
+                out[bi, h, tri_offset(I):tri_offset(I + 1)] = xattn_estimate_block_row(
+                    q[bi, h], kh, I, block, stride, scale)
     return out
 
 

@@ -30,6 +30,9 @@ MUTATIONS = {
                       "return (qhat @ kbar[: (I + 1) * m].T)"),
     "sampled rows reversed": ("qhat = q[rows].astype(np.float64)",
                               "qhat = q[rows].astype(np.float64)[::-1]"),
+    "xattn main diagonal": ("z += qs[:, t, :] @ ks[:, stride - 1 - t, :].T",
+                            "z += qs[:, t, :] @ ks[:, t, :].T"),
+    "xattn scale dropped": ("    return scale * z\n", "    return z\n"),
 }
 
 

@@ -248,3 +248,56 @@ def test_select_tau_one_and_layout():
             row = idx[0, h, orc.tri_offset(I):orc.tri_offset(I + 1)]
             n = cnt[0, h, I]
             assert (np.diff(row[:n]) > 0).all() and row[n - 1] == I and (row[n:] == -1).all()
+
+
+# ---------------------------------------------------------------- XAttention antidiagonal estimator
+
+def test_xattn_stride1_equals_exact_block_softmax_mass():
+    """At S = 1 the antidiagonal of a 1x1 sub-block is the logit itself: the XAttention masses
+    equal the exact block sums of the dense causal softmax (torch fp64), GQA 4:2."""
+    b, hq, hkv, L, d, B = 1, 4, 2, 256, 16, 32
+    q, k = _rand((b, hq, L, d), 30, 0.4), _rand((b, hkv, L, d), 31, 0.4)
+    A = orc.xattn_estimate(q, k, B, 1, 0.8)
+    nb = L // B
+    kt = torch.from_numpy(k).repeat_interleave(hq // hkv, dim=1)
+    s = 0.8 * torch.from_numpy(q) @ kt.transpose(-1, -2)
+    s = s.masked_fill(~torch.ones(L, L, dtype=torch.bool).tril(), float("-inf"))
+    exact = torch.softmax(s, dim=-1).numpy().reshape(b, hq, nb, B, nb, B).sum(axis=(3, 5)) / B
+    for h in range(hq):
+        assert np.abs(_unpack_rows(A[0, h], nb) - exact[0, h]).max() < 1e-12
+
+
+def test_xattn_stride_constant_queries_reduce_to_pooled_keys():
+    """Queries constant inside every stride (Q[iS+t] = c_i) turn the antidiagonal sum into
+    c_i . sum_t K[jS+t]: the masses are the block sums of torch's causal softmax of
+    scale * c_i . Kbar_j."""
+    b, hq, hkv, L, d, B, S, scale = 1, 2, 1, 64, 8, 16, 4, 0.3
+    c = _rand((b, hq, L // S, d), 32)
+    q = np.repeat(c, S, axis=2)
+    k = _rand((b, hkv, L, d), 33)
+    A = orc.xattn_estimate(q, k, B, S, scale)
+    m, nb, ns = B // S, L // B, L // S
+    kbar = k[0, 0].reshape(ns, S, d).sum(axis=1)
+    for h in range(hq):
+        z = torch.from_numpy(scale * c[0, h] @ kbar.T)
+        z = z.masked_fill(~torch.ones(ns, ns, dtype=torch.bool).tril(), float("-inf"))
+        want = torch.softmax(z, dim=-1).numpy().reshape(nb, m, nb, m).sum(axis=(1, 3)) / m
+        assert np.abs(_unpack_rows(A[0, h], nb) - want).max() < 1e-12
+
+
+def test_xattn_direction_is_the_antidiagonal():
+    """Only in-stride query offset 0 carries a query vector and only in-stride key offset S-1
+    carries a key vector, so only the antidiagonal pairing (t, S-1-t) = (0, S-1) sees them:
+    the masses equal the block sums of torch's softmax of scale * Q[iS] . K[jS+S-1]; the main
+    diagonal pairing (t, t) would see zeros everywhere (uniform masses)."""
+    b, hq, hkv, L, d, B, S, scale = 1, 1, 1, 64, 8, 16, 4, 1.0
+    q = np.zeros((b, hq, L, d))
+    k = np.zeros((b, hkv, L, d))
+    q[0, 0, 0::S] = _rand((L // S, d), 34)
+    k[0, 0, S - 1::S] = _rand((L // S, d), 35)
+    A = orc.xattn_estimate(q, k, B, S, scale)
+    m, nb, ns = B // S, L // B, L // S
+    z = torch.from_numpy(scale * q[0, 0, 0::S] @ k[0, 0, S - 1::S].T)
+    z = z.masked_fill(~torch.ones(ns, ns, dtype=torch.bool).tril(), float("-inf"))
+    want = torch.softmax(z, dim=-1).numpy().reshape(nb, m, nb, m).sum(axis=(1, 3)) / m
+    assert np.abs(_unpack_rows(A[0, 0], nb) - want).max() < 1e-12
