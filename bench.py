@@ -447,6 +447,62 @@ def run_speedup_study(args):
     return 0
 
 
+def run_search_study(args):
+    """Pattern-search time: the round-robin estimate (stride pooling + estimate) against the
+    XAttention antidiagonal estimate, both followed by the same select; per length."""
+    import torch
+
+    from long_context_prefill_rr_b200 import native
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    native.load()
+    for L in [int(x) for x in args.lengths.split(",")]:
+        w = wl.WORKLOADS["llama128k"].with_(seqlen=L, name=f"llama{L // 1024}k")
+        q_bits, k_bits, _ = wl.make_workload(w)
+        to = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+        q, k = to(q_bits), to(k_bits)
+        res = {"seq_len": L, "stride": w.stride}
+        p = native.params(w.batch, w.heads_q, w.heads_kv, L, w.head_dim, w.stride, w.tau,
+                          shift=w.shift, softmax_scale=w.softmax_scale)
+        sh = native.shapes(p)
+        mass = torch.empty(sh["mass"], dtype=torch.float32, device=dev)
+        idx = torch.empty(sh["kept_idx"], dtype=torch.int32, device=dev)
+        cnt = torch.empty(sh["kept_cnt"], dtype=torch.int32, device=dev)
+        ws = native.new_workspace(p, dev)
+        for name, fn in (("rr", lambda: native.estimate(p, q, k, mass, ws)),
+                         ("xattn", lambda: native.estimate_xattn(p, q, k, mass, ws))):
+            for _ in range(3):
+                fn()
+                native.select(p, mass, idx, cnt)
+            torch.cuda.synchronize()
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            n = 10
+            t_est = t_sel = 0.0
+            for _ in range(n):
+                e0.record()
+                fn()
+                e1.record()
+                native.select(p, mass, idx, cnt)
+                e2.record()
+                torch.cuda.synchronize()
+                t_est += e0.elapsed_time(e1)
+                t_sel += e1.elapsed_time(e2)
+            st, raw = native.check_device_status(ws)
+            if st != 0:
+                raise RuntimeError(f"device status {raw:#x}")
+            nb = L // 128
+            res[f"{name}_estimate_ms"] = t_est / n
+            res[f"{name}_select_ms"] = t_sel / n
+            res[f"{name}_density"] = float(cnt.sum().item() / (w.heads_q * nb * (nb + 1) / 2))
+        res["xattn_over_rr_search_time"] = ((res["xattn_estimate_ms"] + res["xattn_select_ms"]) /
+                                            (res["rr_estimate_ms"] + res["rr_select_ms"]))
+        print(json.dumps({"study": "search", "workload": w.name, **res}), flush=True)
+        del q, k, mass, idx, cnt, ws
+        torch.cuda.empty_cache()
+    return 0
+
+
 # bump when the attention kernel changes, so stale ncu traffic is not reported
 KERNEL_REV = "attn-v2"
 
@@ -460,12 +516,14 @@ def main(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=12)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--study", choices=["speedup"], default=None,
+    ap.add_argument("--study", choices=["speedup", "search"], default=None,
                     help="instead of the bench line: dense-vs-sparse speedup over --lengths")
     ap.add_argument("--lengths", default="8192,16384,32768,65536,131072")
     args = ap.parse_args(argv)
     if args.study == "speedup":
         return run_speedup_study(args)
+    if args.study == "search":
+        return run_search_study(args)
     w = wl.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

@@ -80,6 +80,17 @@ size_t rra_workspace_bytes(const rra_params *p);
 rra_status rra_estimate(const rra_params *p, const void *q, const void *k, float *mass,
                         void *workspace, size_t workspace_bytes, rra_stream_t stream);
 
+/* Step 1, alternative estimator (the XAttention review, sections 2-3: antidiagonal scoring
+ * with stride-level softmax): the same mass output and layout as rra_estimate, but the
+ * stride-level score of query stride i against key stride j is the sum of the S logits on the
+ * antidiagonal of that S x S sub-block, sum_{t<S} q_{iS+t} . k_{jS+S-1-t}, every head scoring
+ * all of its queries (params->shift is ignored). Causal softmax over strides j <= i and block
+ * sums as in rra_estimate; select and attention are unchanged. Same workspace as rra_estimate.
+ * It costs S times the estimate's tensor-core work, and provides the comparison point for the
+ * pattern-search time. */
+rra_status rra_estimate_xattn(const rra_params *p, const void *q, const void *k, float *mass,
+                              void *workspace, size_t workspace_bytes, rra_stream_t stream);
+
 /* Step 2 (select). mass: fp32 [b, Hq, NB(NB+1)/2] (any non-negative values; negative or NaN
  * entries count as 0). For each row: sort J descending by mass (ties: smaller J first), keep the
  * shortest prefix whose running sum, accumulated in fp64, reaches tau * (fp64 row sum), add the

@@ -7,6 +7,12 @@
 //                         causal (j <= i) stride softmax, block masses
 //                         A[h, I, J] = (1/m) sum_{i in I} sum_{j in J} P[h, i, j].
 //
+// The same kernel, instantiated with XA = true, computes the XAttention antidiagonal estimate
+// (XAttention review, sections 2-3): the logit tile is sum_{t<S} Q_t . K_{S-1-t}^T, where Q_t
+// holds the queries at in-stride offset t of 128 query strides and K_{S-1-t} the keys at offset
+// S-1-t of 128 key strides; the S products accumulate into one TMEM tile (exact bf16 operands,
+// no pooling, no hi/lo split), and the epilogue is the same.
+//
 // K2 is a persistent, warp-specialised kernel. One work item is (batch, head, tile of 128
 // sampled queries); the CTA streams the 128-stride key tiles n = 0..t through a 2-stage TMA
 // ring, the MMA warp computes each 128x128 logit tile into one of two TMEM accumulators as
@@ -88,7 +94,9 @@ __device__ __forceinline__ void est_decode(const EstParams &p, int item, int &bh
   t = p.ntiles - 1 - level;
 }
 
-template <int D, int M>
+// RR: tm_q = 3-D view of Q (box at in-stride offset o_h), tm_khi / tm_klo = pooled keys.
+// XA: tm_q = the same 3-D view of Q, tm_khi = 3-D view of K (box at in-stride offset S-1-t).
+template <int D, int M, bool XA>
 __global__ void __launch_bounds__(384, 1)
     rr_estimate_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_khi,
@@ -96,7 +104,9 @@ __global__ void __launch_bounds__(384, 1)
   constexpr int NCHUNK = D / 64;                  // 64-column (128-byte) chunks per row
   constexpr uint32_t CHUNK_BYTES = 128 * 128;     // 128 rows x 128 bytes
   constexpr uint32_t TILE_BYTES = NCHUNK * CHUNK_BYTES;
-  constexpr int NSTAGE = 2;
+  // RR: resident sampled-query tile + 2 stages of (Kbar hi, Kbar lo); XA: 3 stages of (Q_t, K_t)
+  constexpr int NSTAGE = XA ? 3 : 2;
+  constexpr uint32_t Q_RES = XA ? 0 : TILE_BYTES;
   constexpr int SEG = 64 / M;                     // key blocks per 64-column half tile
   constexpr int SEG_ROW = 128 / M;                // key blocks per 128-stride key tile
   constexpr uint32_t IDESC = idesc_bf16_f32(128, 128, false);
@@ -105,16 +115,16 @@ __global__ void __launch_bounds__(384, 1)
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t *sQ = smem;
-  uint8_t *sK = smem + TILE_BYTES;                // stage s: hi at s*2*TILE, lo at +TILE
+  uint8_t *sK = smem + Q_RES;                     // stage s at s*2*TILE: (hi, lo) or (Q_t, K_t)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sK + NSTAGE * 2 * TILE_BYTES);
   uint64_t *q_full = bars + 0;
   uint64_t *q_empty = bars + 1;
   uint64_t *kv_full = bars + 2;                   // [NSTAGE]
-  uint64_t *kv_empty = bars + 4;                  // [NSTAGE]
-  uint64_t *acc_full = bars + 6;                  // [2]
-  uint64_t *acc_empty = bars + 8;                 // [2]
-  uint64_t *drain = bars + 10;
-  float *sM = reinterpret_cast<float *>(bars + 12);   // [2][128]
+  uint64_t *kv_empty = kv_full + NSTAGE;          // [NSTAGE]
+  uint64_t *acc_full = kv_empty + NSTAGE;         // [2]
+  uint64_t *acc_empty = acc_full + 2;             // [2]
+  uint64_t *drain = acc_empty + 2;
+  float *sM = reinterpret_cast<float *>(drain + 2);   // [2][128]
   float *sL = sM + 256;                               // [2][128]
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sL + 256);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
@@ -159,7 +169,8 @@ __global__ void __launch_bounds__(384, 1)
       int stage = 0;
       uint32_t phase = 0, qph = 0;
       int issued_q = 0;
-      int issued[NSTAGE] = {0, 0};
+      int issued[NSTAGE];
+      for (int s2 = 0; s2 < NSTAGE; ++s2) issued[s2] = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         int bh, t;
@@ -168,6 +179,32 @@ __global__ void __launch_bounds__(384, 1)
         const int b = bh / p.hq;
         const int kv = h / p.g;
         const int o = ((h + p.shift) % p.S + p.S) % p.S;
+        const int krow = (b * p.hkv + kv) * p.ns;
+        if constexpr (XA) {
+          // per key tile: S stages of (queries at offset tt, keys at offset S-1-tt)
+          for (int n = 0; n <= t && ok; ++n)
+            for (int tt = 0; tt < p.S; ++tt) {
+              if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) {
+                ok = false;
+                break;
+              }
+              mbar_arrive_expect_tx(&kv_full[stage], 2 * TILE_BYTES);
+              uint8_t *st = sK + stage * 2 * TILE_BYTES;
+              for (int c = 0; c < NCHUNK; ++c) {
+                tma_load_3d(st + c * CHUNK_BYTES, &tm_q, &kv_full[stage], c * 64, tt,
+                            bh * p.ns + t * 128);
+                tma_load_3d(st + TILE_BYTES + c * CHUNK_BYTES, &tm_khi, &kv_full[stage],
+                            c * 64, p.S - 1 - tt, krow + n * 128);
+              }
+              ++issued[stage];
+              if (++stage == NSTAGE) {
+                stage = 0;
+                phase ^= 1;
+              }
+            }
+          (void)o;
+          continue;
+        }
         if (issued_q > 0) {
           if (!mbar_wait(q_empty, qph, s_abort, p.status)) break;
           qph ^= 1;
@@ -176,7 +213,6 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < NCHUNK; ++c)
           tma_load_3d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, o, bh * p.ns + t * 128);
         ++issued_q;
-        const int krow = (b * p.hkv + kv) * p.ns;
         for (int n = 0; n <= t; ++n) {
           if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) {
             ok = false;
@@ -213,6 +249,44 @@ __global__ void __launch_bounds__(384, 1)
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         int bh, t;
         est_decode(p, item, bh, t);
+        if constexpr (XA) {
+          for (int n = 0; n <= t && ok; ++n) {
+            if (!mbar_wait(&acc_empty[acc], aph ^ 1, s_abort, p.status)) {
+              ok = false;
+              break;
+            }
+            const uint32_t d_tmem = tmem + acc * 128;
+            for (int tt = 0; tt < p.S; ++tt) {
+              if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint32_t a_base = smem_u32(sK + stage * 2 * TILE_BYTES);
+              const uint32_t b_base = a_base + TILE_BYTES;
+#pragma unroll
+              for (int c = 0; c < NCHUNK; ++c)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                  const uint64_t a = sdesc_kmajor_sw128(a_base + c * CHUNK_BYTES + kk * 32);
+                  const uint64_t bd = sdesc_kmajor_sw128(b_base + c * CHUNK_BYTES + kk * 32);
+                  mma_bf16_ss(d_tmem, a, bd, IDESC, (tt | c | kk) != 0);
+                }
+              mma_commit(&kv_empty[stage]);
+              if (++stage == NSTAGE) {
+                stage = 0;
+                phase ^= 1;
+              }
+            }
+            if (!ok) break;
+            mma_commit(&acc_full[acc]);
+            if (++acc == 2) {
+              acc = 0;
+              aph ^= 1;
+            }
+          }
+          continue;
+        }
         if (!mbar_wait(q_full, qph, s_abort, p.status)) break;
         qph ^= 1;
         for (int n = 0; n <= t; ++n) {
@@ -444,13 +518,15 @@ cudaError_t launch_pool_keys(const Geometry &g, const void *k, void *khi, void *
   return cudaGetLastError();
 }
 
-template <int D, int M>
+template <int D, int M, bool XA>
 static cudaError_t launch_est_t(const CUtensorMap &mq, const CUtensorMap &mhi,
                                 const CUtensorMap &mlo, const EstParams &ep, int slots,
                                 cudaStream_t stream) {
   constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
-  const size_t smem = 1024 + TILE * (1 + 2 * 2) + 12 * 8 + 512 * 4 + 16;
-  auto kern = rr_estimate_kernel<D, M>;
+  constexpr int NSTAGE = XA ? 3 : 2;
+  const size_t smem = 1024 + TILE * ((XA ? 0 : 1) + 2 * NSTAGE) + (2 + 2 * NSTAGE + 6) * 8 +
+                      512 * 4 + 16;
+  auto kern = rr_estimate_kernel<D, M, XA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -458,23 +534,40 @@ static cudaError_t launch_est_t(const CUtensorMap &mq, const CUtensorMap &mhi,
   return cudaGetLastError();
 }
 
-cudaError_t launch_rr_estimate(const Geometry &g, const void *q, const void *khi,
-                               const void *klo, float *mass, float *est_e, float *est_ref,
-                               int slots, uint32_t *status, cudaStream_t stream) {
-  CUtensorMap mq, mhi, mlo;
-  const cuuint64_t bhq_ns = static_cast<cuuint64_t>(g.b) * g.hq * g.ns;
-  const cuuint64_t qdims[3] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.S), bhq_ns};
-  const cuuint64_t qstr[2] = {static_cast<cuuint64_t>(g.d) * 2,
-                              static_cast<cuuint64_t>(g.S) * g.d * 2};
-  const cuuint32_t qbox[3] = {64, 1, 128};
-  if (!make_map(&mq, const_cast<void *>(q), 3, qdims, qstr, qbox)) return cudaErrorInvalidValue;
-  const cuuint64_t kdims[2] = {static_cast<cuuint64_t>(g.d),
-                               static_cast<cuuint64_t>(g.b) * g.hkv * g.ns};
-  const cuuint64_t kstr[1] = {static_cast<cuuint64_t>(g.d) * 2};
-  const cuuint32_t kbox[2] = {64, 128};
-  if (!make_map(&mhi, const_cast<void *>(khi), 2, kdims, kstr, kbox)) return cudaErrorInvalidValue;
-  if (!make_map(&mlo, const_cast<void *>(klo), 2, kdims, kstr, kbox)) return cudaErrorInvalidValue;
+template <bool XA>
+static cudaError_t dispatch_est(const Geometry &g, const CUtensorMap &mq, const CUtensorMap &mhi,
+                                const CUtensorMap &mlo, const EstParams &ep, int slots,
+                                cudaStream_t stream) {
+  if (g.d == 128) {
+    switch (g.m) {
+      case 4: return launch_est_t<128, 4, XA>(mq, mhi, mlo, ep, slots, stream);
+      case 8: return launch_est_t<128, 8, XA>(mq, mhi, mlo, ep, slots, stream);
+      case 16: return launch_est_t<128, 16, XA>(mq, mhi, mlo, ep, slots, stream);
+      case 32: return launch_est_t<128, 32, XA>(mq, mhi, mlo, ep, slots, stream);
+    }
+  } else if (g.d == 64) {
+    switch (g.m) {
+      case 4: return launch_est_t<64, 4, XA>(mq, mhi, mlo, ep, slots, stream);
+      case 8: return launch_est_t<64, 8, XA>(mq, mhi, mlo, ep, slots, stream);
+      case 16: return launch_est_t<64, 16, XA>(mq, mhi, mlo, ep, slots, stream);
+      case 32: return launch_est_t<64, 32, XA>(mq, mhi, mlo, ep, slots, stream);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
 
+// 3-D view (d, S, rows / S) of a [rows, d] bf16 tensor: a {64, 1, 128} box at in-stride offset
+// o picks 128 rows spaced S apart.
+static bool make_strided_map(CUtensorMap *map, const void *base, int64_t rows, int d, int S) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(S),
+                              static_cast<cuuint64_t>(rows / S)};
+  const cuuint64_t str[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(S) * d * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
+  return make_map(map, const_cast<void *>(base), 3, dims, str, box);
+}
+
+static EstParams est_params(const Geometry &g, float *mass, float *est_e, float *est_ref,
+                            uint32_t *status) {
   EstParams ep;
   ep.hq = g.hq;
   ep.hkv = g.hkv;
@@ -491,23 +584,36 @@ cudaError_t launch_rr_estimate(const Geometry &g, const void *q, const void *khi
   ep.est_e = est_e;
   ep.est_ref = est_ref;
   ep.status = status;
+  return ep;
+}
+
+cudaError_t launch_rr_estimate(const Geometry &g, const void *q, const void *khi,
+                               const void *klo, float *mass, float *est_e, float *est_ref,
+                               int slots, uint32_t *status, cudaStream_t stream) {
+  CUtensorMap mq, mhi, mlo;
+  if (!make_strided_map(&mq, q, static_cast<int64_t>(g.b) * g.hq * g.L, g.d, g.S))
+    return cudaErrorInvalidValue;
+  const cuuint64_t kdims[2] = {static_cast<cuuint64_t>(g.d),
+                               static_cast<cuuint64_t>(g.b) * g.hkv * g.ns};
+  const cuuint64_t kstr[1] = {static_cast<cuuint64_t>(g.d) * 2};
+  const cuuint32_t kbox[2] = {64, 128};
+  if (!make_map(&mhi, const_cast<void *>(khi), 2, kdims, kstr, kbox)) return cudaErrorInvalidValue;
+  if (!make_map(&mlo, const_cast<void *>(klo), 2, kdims, kstr, kbox)) return cudaErrorInvalidValue;
+  const EstParams ep = est_params(g, mass, est_e, est_ref, status);
   if (slots > ep.n_items) slots = ep.n_items;
-  if (g.d == 128) {
-    switch (g.m) {
-      case 4: return launch_est_t<128, 4>(mq, mhi, mlo, ep, slots, stream);
-      case 8: return launch_est_t<128, 8>(mq, mhi, mlo, ep, slots, stream);
-      case 16: return launch_est_t<128, 16>(mq, mhi, mlo, ep, slots, stream);
-      case 32: return launch_est_t<128, 32>(mq, mhi, mlo, ep, slots, stream);
-    }
-  } else if (g.d == 64) {
-    switch (g.m) {
-      case 4: return launch_est_t<64, 4>(mq, mhi, mlo, ep, slots, stream);
-      case 8: return launch_est_t<64, 8>(mq, mhi, mlo, ep, slots, stream);
-      case 16: return launch_est_t<64, 16>(mq, mhi, mlo, ep, slots, stream);
-      case 32: return launch_est_t<64, 32>(mq, mhi, mlo, ep, slots, stream);
-    }
-  }
-  return cudaErrorInvalidValue;
+  return dispatch_est<false>(g, mq, mhi, mlo, ep, slots, stream);
+}
+
+cudaError_t launch_xattn_estimate(const Geometry &g, const void *q, const void *k, float *mass,
+                                  float *est_e, float *est_ref, int slots, uint32_t *status,
+                                  cudaStream_t stream) {
+  CUtensorMap mq, mk;
+  if (!make_strided_map(&mq, q, static_cast<int64_t>(g.b) * g.hq * g.L, g.d, g.S) ||
+      !make_strided_map(&mk, k, static_cast<int64_t>(g.b) * g.hkv * g.L, g.d, g.S))
+    return cudaErrorInvalidValue;
+  const EstParams ep = est_params(g, mass, est_e, est_ref, status);
+  if (slots > ep.n_items) slots = ep.n_items;
+  return dispatch_est<true>(g, mq, mk, mk, ep, slots, stream);
 }
 
 }  // namespace rra

@@ -156,6 +156,22 @@ rra_status rra_estimate(const rra_params *p, const void *q, const void *k, float
   return run_estimate(g, q, k, mass, workspace, w, sms, reinterpret_cast<cudaStream_t>(stream));
 }
 
+rra_status rra_estimate_xattn(const rra_params *p, const void *q, const void *k, float *mass,
+                              void *workspace, size_t workspace_bytes, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, kNeedsStride | kNeedsHeadDim, &g);
+  if (s != RRA_OK) return s;
+  if (empty(g)) return RRA_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(mass) || !ptr_ok(workspace)) return RRA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return RRA_ERR_CUDA;
+  const WorkspaceLayout w = rra::workspace_layout(g, sms);
+  if (workspace_bytes < w.total) return RRA_ERR_WORKSPACE;
+  return cuda_status(rra::launch_xattn_estimate(
+      g, q, k, mass, ws_at<float>(workspace, w.est_e), ws_at<float>(workspace, w.est_ref),
+      w.est_slots, status_word(workspace, w), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rra_status rra_select(const rra_params *p, const float *mass, int32_t *kept_idx,
                       int32_t *kept_cnt, rra_stream_t stream) {
   Geometry g;

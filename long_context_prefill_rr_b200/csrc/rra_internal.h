@@ -47,6 +47,9 @@ cudaError_t launch_pool_keys(const Geometry &g, const void *k, void *khi, void *
 cudaError_t launch_rr_estimate(const Geometry &g, const void *q, const void *khi,
                                const void *klo, float *mass, float *est_e, float *est_ref,
                                int slots, uint32_t *status, cudaStream_t stream);
+cudaError_t launch_xattn_estimate(const Geometry &g, const void *q, const void *k, float *mass,
+                                  float *est_e, float *est_ref, int slots, uint32_t *status,
+                                  cudaStream_t stream);
 cudaError_t launch_topt_select(const Geometry &g, const float *mass, int32_t *kept_idx,
                                int32_t *kept_cnt, int num_sms, cudaStream_t stream);
 cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, const void *v,

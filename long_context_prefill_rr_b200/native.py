@@ -32,6 +32,8 @@ _SIGS = {
     "rra_prefill": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                _c.c_void_p]),
+    "rra_estimate_xattn": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                      _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "rra_estimate_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p,
                                                _c.c_void_p, _c.c_void_p]),
     "rra_check_device_status": (_c.c_int, [_c.c_void_p, _c.c_void_p,
@@ -146,6 +148,17 @@ def estimate(p: RraParams, q, k, mass, ws, stream=None):
     _expect(mass, torch.float32, sh["mass"], "mass")
     _check(load().rra_estimate(_p(p), _ptr(q), _ptr(k), _ptr(mass), _ptr(ws), ws.numel(),
                                _stream(stream)), "rra_estimate")
+
+
+def estimate_xattn(p: RraParams, q, k, mass, ws, stream=None):
+    """XAttention antidiagonal estimate (same mass layout as ``estimate``)."""
+    import torch
+    sh = shapes(p)
+    _expect(q, torch.bfloat16, sh["q"], "q")
+    _expect(k, torch.bfloat16, sh["kv"], "k")
+    _expect(mass, torch.float32, sh["mass"], "mass")
+    _check(load().rra_estimate_xattn(_p(p), _ptr(q), _ptr(k), _ptr(mass), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "rra_estimate_xattn")
 
 
 def estimate_static_scratch(p: RraParams, q, k, mass, stream=None):

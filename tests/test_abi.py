@@ -29,8 +29,8 @@ def lib():
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
         "rra_workspace_bytes", "rra_estimate", "rra_select", "rra_sparse_attn", "rra_prefill",
-        "rra_estimate_static_scratch", "rra_check_device_status", "rra_status_string",
-        "rra_version"])
+        "rra_estimate_static_scratch", "rra_estimate_xattn", "rra_check_device_status",
+        "rra_status_string", "rra_version"])
 
 
 def test_library_exports_every_declared_symbol(lib):
