@@ -6,7 +6,8 @@ One step = one attention layer's prefill: pooled-key estimate, Top-tau select an
 attention (rra_estimate, rra_select, rra_sparse_attn through the C ABI) on the seeded
 Llama-3.1-8B-like layer at 128K tokens (b1, 32 Q / 8 KV heads, d 128, B 128, S 8, tau 0.9).
 Inputs (2.7 GB) are larger than L2, so no flush is needed between steps. With N > 1 (torchrun)
-every rank runs an independent replica of the layer; the time is the max over ranks.
+every rank runs an independent replica of the layer (default), or with --shard heads its share
+of the KV-head groups of one layer (no exchange between ranks); the time is the max over ranks.
 
 Prints one JSON line (rank 0). `value` is milliseconds per layer for the whole job
 (max-over-ranks step time / layers processed per step). The reference arm times the fp64 CPU
@@ -27,6 +28,7 @@ sys.path.insert(0, ROOT)
 
 import numpy as np  # noqa: E402
 
+from long_context_prefill_rr_b200 import sharding  # noqa: E402
 from long_context_prefill_rr_b200 import workloads as wl  # noqa: E402
 
 METRIC = "prefill attn ms/layer @128K (estimate+select+sparse) & TFLOP/s vs roofline"
@@ -43,14 +45,14 @@ def _peaks():
             "source": "fallback"}
 
 
-def _workload_desc(w: wl.Workload) -> dict:
+def _workload_desc(w: wl.Workload, parallelism: str = "replicas") -> dict:
     return {"workload": f"{w.name}: b{w.batch} Hq{w.heads_q} Hkv{w.heads_kv} d{w.head_dim} "
                         f"L{w.seqlen} B{w.block} S{w.stride} tau{w.tau}",
             "model": "Llama-3.1-8B-like attention layer (random synthetic Q/K/V)"
             if w.kind == "llama" else w.kind,
             "global_batch": w.batch, "seq_len": w.seqlen, "heads_q": w.heads_q,
             "heads_kv": w.heads_kv, "head_dim": w.head_dim, "block": w.block, "stride": w.stride,
-            "tau": w.tau, "parallelism": "replicas", "l2": "inputs (2.7 GB) larger than L2"
+            "tau": w.tau, "parallelism": parallelism, "l2": "inputs (2.7 GB) larger than L2"
             if w.seqlen >= 32768 else "L2 flushed between steps"}
 
 
@@ -193,6 +195,16 @@ def max_over_ranks(values, device=None):
     return [float(x) for x in t.cpu()]
 
 
+def sum_over_ranks(values, device=None):
+    """Element-wise sum over the process group (identity when there is none)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.cpu()]
+
+
 def run_reference(args, w):
     ws, rank, _ = _dist_env()
     if rank != 0:
@@ -231,8 +243,15 @@ def run_gpu(args, w):
     native.load()
     p = native.params(w.batch, w.heads_q, w.heads_kv, w.seqlen, w.head_dim, w.stride, w.tau,
                       shift=w.shift, softmax_scale=w.softmax_scale, block=w.block)
-    sh = native.shapes(p)
     q_bits, k_bits, v_bits = wl.make_workload(w)
+    sharded = args.shard == "heads"
+    if sharded:
+        # this rank's KV-head groups; no data moves between ranks on the path
+        p, shard = sharding.shard_params(p, rank, ws_n)
+        q_bits = sharding.take_heads(q_bits, shard.q0, shard.q1)
+        k_bits = sharding.take_heads(k_bits, shard.kv0, shard.kv1)
+        v_bits = sharding.take_heads(v_bits, shard.kv0, shard.kv1)
+    sh = native.shapes(p)
 
     def host_pinned(bits):
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
@@ -306,27 +325,33 @@ def run_gpu(args, w):
     e2e_ms = e_start.elapsed_time(e_stop) / e_steps
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
+    useful, executed, n_kept = attention_flops(idx.cpu().numpy(), cnt.cpu().numpy(), w.block,
+                                               w.head_dim)
+    h2d_bytes = int(hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h_bytes = int(hout.numel()) * 2
+    # whole-job figures: kept blocks over every rank's heads, bytes every rank moved
+    n_kept_all, h2d_all, d2h_all = sum_over_ranks([n_kept, h2d_bytes, d2h_bytes], dev)
 
     if rank == 0:
         peaks = _peaks()
-        kept_idx = idx.cpu().numpy()
-        kept_cnt = cnt.cpu().numpy()
-        useful, executed, n_kept = attention_flops(kept_idx, kept_cnt, w.block, w.head_dim)
         nb = w.seqlen // w.block
-        density = n_kept / (w.batch * w.heads_q * nb * (nb + 1) / 2)
+        heads_all = w.heads_q * (1 if sharded else ws_n)
+        density = n_kept_all / (w.batch * heads_all * nb * (nb + 1) / 2)
         att_avg = float(np.mean(att_ms))
         est_avg = float(np.mean(est_ms))
         sel_avg = float(np.mean(sel_ms))
         achieved = useful / (att_avg * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         ns = w.seqlen // w.stride
-        est_bytes = (w.batch * w.heads_kv * w.seqlen * w.head_dim * 2          # K read once
-                     + w.batch * w.heads_q * ns * w.head_dim * 2               # sampled Q rows
-                     + w.batch * w.heads_q * nb * (nb + 1) // 2 * 4)           # masses out
-        sel_bytes = (w.batch * w.heads_q * nb * (nb + 1) // 2 * 4 + n_kept * 4 +
-                     w.batch * w.heads_q * nb * 4)
+        # per-rank algorithmic bytes (this rank's heads)
+        est_bytes = (p.batch * p.heads_kv * w.seqlen * w.head_dim * 2          # K read once
+                     + p.batch * p.heads_q * ns * w.head_dim * 2               # sampled Q rows
+                     + p.batch * p.heads_q * nb * (nb + 1) // 2 * 4)           # masses out
+        sel_bytes = (p.batch * p.heads_q * nb * (nb + 1) // 2 * 4 + n_kept * 4 +
+                     p.batch * p.heads_q * nb * 4)
         ms_per_step = total_ms / args.steps
-        value = ms_per_step / ws_n
+        # ms per layer of the whole job: replicas finish ws_n layers per step, head shards one
+        value = ms_per_step if sharded else ms_per_step / ws_n
         cpu = None
         if ws_n == 1 and not args.no_cpu_baseline:
             cpu = cpu_oracle_sample(w, q_bits, k_bits, v_bits, n_rows=args.ref_rows,
@@ -340,9 +365,10 @@ def run_gpu(args, w):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": False, "scaling": "strong" if sharded else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded, shaped like the pages' Llama-3.1-8B 128K workload)",
-            "config": _workload_desc(w),
+            "config": _workload_desc(w, f"heads{ws_n}" if sharded else "replicas"),
             "phases_ms": {"estimate": est_avg, "select": sel_avg, "sparse_attn": att_avg},
             "density": density,
             "attn_tflops": achieved, "attn_tflops_executed": executed / (att_avg * 1e-3) / 1e12,
@@ -357,9 +383,8 @@ def run_gpu(args, w):
                          "traffic": traffic,
                          "per_launch_flops": useful},
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_ms / ws_n, "unit": UNIT,
-                    "h2d_bytes_per_step": int(hq.numel() + hk.numel() + hv.numel()) * 2,
-                    "d2h_bytes_per_step": int(hout.numel()) * 2},
+            "e2e": {"value": e2e_ms if sharded else e2e_ms / ws_n, "unit": UNIT,
+                    "h2d_bytes_per_step": int(h2d_all), "d2h_bytes_per_step": int(d2h_all)},
             "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
         }
@@ -504,7 +529,7 @@ def run_search_study(args):
 
 
 # bump when the attention kernel changes, so stale ncu traffic is not reported
-KERNEL_REV = "attn-v2"
+KERNEL_REV = "attn-v3"
 
 
 def main(argv=None):
@@ -519,6 +544,9 @@ def main(argv=None):
     ap.add_argument("--study", choices=["speedup", "search"], default=None,
                     help="instead of the bench line: dense-vs-sparse speedup over --lengths")
     ap.add_argument("--lengths", default="8192,16384,32768,65536,131072")
+    ap.add_argument("--shard", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: every rank runs the whole layer (replicas, weak scaling) or "
+                         "its share of the KV-head groups (heads, strong scaling)")
     args = ap.parse_args(argv)
     if args.study == "speedup":
         return run_speedup_study(args)

@@ -3,19 +3,23 @@
 // digest; online softmax as in FlashAttention / FlashAttention-2), GQA head mapping.
 //
 // One CTA runs two work items side by side: query block I of heads 2c and 2c+1 (of one batch
-// row), each with its own kept list. Grid order is longest-first (I descending). Roles:
+// row), each with its own kept list. Grid order is by KV-head chunk, then longest-first (I
+// descending) within the chunk (see attn_item). Roles:
 //   warp 0       TMA producer: both Q tiles once, then per step j the tiles V_A(j-1), K_A(j),
 //                V_B(j-1), K_B(j) through a ring of 128-row tiles, in the order the MMA warp
 //                consumes them;
 //   warp 1       MMA issuer (one thread), same order: O_X += P_X V_X(j-1) with P read from TMEM
-//                (tcgen05 "TS" form), then S_X = Q_X K_X(j)^T into the same TMEM columns. While
-//                one item's softmax runs, the tensor core works on the other item (ping-pong);
+//                (tcgen05 "TS" form; keys 0..63 as soon as that half of P is written, keys
+//                64..127 when the rest is), then S_X = Q_X K_X(j)^T into the same TMEM columns.
+//                While one item's softmax runs, the tensor core works on the other item
+//                (ping-pong). The warp counts each item's valid tiles up front, so its issue
+//                loop reads no global memory;
 //   warp 2       TMEM allocation: S/P_A | S/P_B | O_A | O_B (512 columns for d = 128);
 //   warps 4-7    softmax of item A, warps 8-11 softmax of item B: one thread per query row reads
 //                its 128 logits from TMEM, masks the diagonal block, keeps a running max (O is
-//                rescaled in TMEM only when the max grows by more than 2^8, decided per warp)
-//                and running sum, writes P as bf16 back over S, and at the end normalises O
-//                and stores the bf16 row.
+//                rescaled in TMEM, before any P of the tile is published, only when the max
+//                grows by more than 2^8, decided per warp) and running sum, writes P as bf16
+//                back over S in two halves, and at the end normalises O and stores the bf16 row.
 // Because the S/P columns of an item are reused every tile, S_X(j) completing implies the
 // previous PV product of that item completed (MMAs complete in issue order), so O_X is stable
 // whenever its softmax runs.
@@ -31,6 +35,7 @@ namespace rra {
 struct AttnParams {
   int hq, hkv, g, L, nb, batch;
   int n_pairs;       // batch * ceil(hq / 2)
+  int chunk;         // head pairs per KV-head chunk of the launch order (ceil(g / 2))
   int64_t tri;
   float scale_log2;
   const int32_t *kept_idx;
@@ -39,10 +44,11 @@ struct AttnParams {
   uint32_t *status;
 };
 
-// Walks one kept row, yielding the valid entries (0 <= J <= I, strictly ascending).
+// Walks one kept row, yielding the valid entries (0 <= J <= I, strictly ascending). The entry
+// after the current one is loaded one call ahead, so its latency overlaps the caller's work.
 struct ListCursor {
   const int32_t *lst;
-  int cnt, e, prev, I;
+  int cnt, e, prev, I, ahead;
   __device__ void init(const AttnParams &p, int bh, int I_, bool valid) {
     I = I_;
     e = 0;
@@ -54,11 +60,13 @@ struct ListCursor {
       if (cnt < 0) cnt = 0;
       if (cnt > I + 1) cnt = I + 1;
     }
+    ahead = cnt > 0 ? lst[0] : -1;
   }
   // next valid block index, or -1; invalid entries are reported through `status` if non-null
   __device__ int next(uint32_t *status) {
     while (e < cnt) {
-      const int J = lst[e++];
+      const int J = ahead;
+      if (++e < cnt) ahead = lst[e];
       if (J > prev && J <= I) {
         prev = J;
         return J;
@@ -68,6 +76,61 @@ struct ListCursor {
     return -1;
   }
 };
+
+// Number of entries ListCursor::next yields for one row, counted by a whole warp: an entry is
+// yielded iff it lies in [0, I] and exceeds every earlier in-range entry (the yielded entries
+// are then the strict running maxima of the in-range ones).
+__device__ int count_valid_warp(const AttnParams &p, int bh, int I, bool valid, int lane) {
+  if (!valid) return 0;
+  int cnt = p.kept_cnt[static_cast<int64_t>(bh) * p.nb + I];
+  cnt = cnt < 0 ? 0 : (cnt > I + 1 ? I + 1 : cnt);
+  const int32_t *lst =
+      p.kept_idx + static_cast<int64_t>(bh) * p.tri + static_cast<int64_t>(I) * (I + 1) / 2;
+  int carry = -1, n = 0;
+  for (int base = 0; base < cnt; base += 32) {
+    const int e = base + lane;
+    const int J = e < cnt ? lst[e] : -1;
+    const int v = (J >= 0 && J <= I) ? J : -1;
+    int pm = v;   // inclusive prefix max over the chunk
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, pm, off);
+      if (lane >= off) pm = max(pm, o);
+    }
+    int before = __shfl_up_sync(0xffffffffu, pm, 1);
+    before = lane == 0 ? carry : max(before, carry);
+    n += __popc(__ballot_sync(0xffffffffu, v >= 0 && v > before));
+    carry = max(carry, __shfl_sync(0xffffffffu, pm, 31));
+  }
+  return n;
+}
+
+// Launch order: per batch row, chunks of `chunk` head pairs (the query heads of about one KV
+// head), each chunk's block rows longest first (I descending), the chunk's pairs innermost. The
+// CTAs resident at one time then read the K/V tiles of one or two KV heads, which fit in L2 even
+// at long lengths, so a tile kept by several rows or heads is fetched from DRAM about once.
+__device__ __forceinline__ void attn_item(const AttnParams &p, int64_t idx, int &b, int &c,
+                                          int &level) {
+  const int hp = (p.hq + 1) >> 1;
+  const int64_t per_b = static_cast<int64_t>(p.nb) * hp;
+  b = static_cast<int>(idx / per_b);
+  const int64_t r = idx - b * per_b;
+  const int C = p.chunk;
+  const int nfull = hp / C;
+  const int64_t full = static_cast<int64_t>(nfull) * p.nb * C;
+  if (r < full) {
+    const int64_t per_chunk = static_cast<int64_t>(p.nb) * C;
+    const int k = static_cast<int>(r / per_chunk);
+    const int64_t s = r - k * per_chunk;
+    level = static_cast<int>(s / C);
+    c = k * C + static_cast<int>(s - static_cast<int64_t>(level) * C);
+  } else {   // the last, narrower chunk
+    const int crem = hp - nfull * C;
+    const int64_t s = r - full;
+    level = static_cast<int>(s / crem);
+    c = nfull * C + static_cast<int>(s - static_cast<int64_t>(level) * crem);
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(384, 1)
@@ -93,19 +156,18 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t *kv_empty = kv_full + NSTAGE;            // [NSTAGE]
   uint64_t *s_full = kv_empty + NSTAGE;             // [2]
   uint64_t *p_full = s_full + 2;                    // [2]
-  uint64_t *o_final = p_full + 2;                   // [2]
+  uint64_t *p_half = p_full + 2;                    // [2] P of keys 0..63 written
+  uint64_t *o_final = p_half + 2;                   // [2]
   uint64_t *drain = o_final + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int level = blockIdx.x / p.n_pairs;
-  const int pair = blockIdx.x - level * p.n_pairs;
+  int b, c, level;
+  attn_item(p, blockIdx.x, b, c, level);
   const int I = p.nb - 1 - level;
-  const int hp = (p.hq + 1) >> 1;
-  const int b = pair / hp;
-  const int h0 = 2 * (pair - b * hp);
+  const int h0 = 2 * c;
   int bh[2], kvrow[2];
   bool valid[2];
 #pragma unroll
@@ -126,6 +188,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
       mbar_init(&p_full[x], 128);
+      mbar_init(&p_half[x], 128);
       mbar_init(&o_final[x], 1);
     }
     mbar_init(drain, 1);
@@ -210,67 +273,68 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Tile counts first (whole warp), so the issue loop itself touches no global memory.
+    int n[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) n[x] = count_valid_warp(p, bh[x], I, valid[x], lane);
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      bool ok = true, q_ready = false;
-      const uint32_t q_base = smem_u32(sQ);
-      ListCursor cur[2];
-      int J[2], ntile[2] = {0, 0};
-      bool pend[2] = {false, false};
-      for (int x = 0; x < 2; ++x) {
-        cur[x].init(p, bh[x], I, valid[x]);
-        J[x] = cur[x].next(nullptr);
-      }
-      while (ok) {
-        bool any = false;
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (pend[x]) {
-            // O_x += P_x(t) V_x(t), t = ntile[x] - 1; P sits in the S columns of item x
-            const int t = ntile[x] - 1;
-            if (!mbar_wait(&p_full[x], t & 1, s_abort, p.status) ||
+      bool ok = true;
+      if (n[0] + n[1] > 0) ok = mbar_wait(q_full, 0, s_abort, p.status);
+      // descriptors: base of each operand; per-MMA offsets are added in 16-byte units
+      const uint32_t ring_base = smem_u32(sRing);
+      const uint64_t q_desc[2] = {sdesc_kmajor_sw128(smem_u32(sQ)),
+                                  sdesc_kmajor_sw128(smem_u32(sQ) + TILE_BYTES)};
+      const uint64_t k_desc0 = sdesc_kmajor_sw128(ring_base);
+      const uint64_t v_desc0 = sdesc_mnmajor_sw128(ring_base, CHUNK_BYTES);
+      const int steps = max(n[0], n[1]);
+      for (int j = 0; j <= steps && ok; ++j) {
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+          if (j >= 1 && j <= n[x]) {
+            // O_x += P_x(j-1) V_x(j-1); P sits in the S columns of item x. Keys 0..63 go in
+            // as soon as their half of P is written, while the softmax finishes keys 64..127.
+            if (!mbar_wait(&p_half[x], (j - 1) & 1, s_abort, p.status) ||
                 !mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t v_base = smem_u32(sRing + stage * TILE_BYTES);
+            const uint64_t vd = v_desc0 + ((stage * TILE_BYTES) >> 4);
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t bd = sdesc_mnmajor_sw128(v_base + kk * 2048, CHUNK_BYTES);
-              mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, bd, IDESC_O, (t > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
+                          (j > 1 || kk > 0) ? 1u : 0u);
+            if (!mbar_wait(&p_full[x], (j - 1) & 1, s_abort, p.status)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4; kk < 8; ++kk)
+              mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, vd + kk * (2048 >> 4), IDESC_O, 1u);
             mma_commit(&kv_empty[stage]);
-            if (J[x] < 0) mma_commit(&o_final[x]);
+            if (j == n[x]) mma_commit(&o_final[x]);
             if (++stage == NSTAGE) {
               stage = 0;
               phase ^= 1;
             }
-            pend[x] = false;
-            any = true;
           }
-          if (J[x] >= 0) {
-            if (!q_ready) {
-              if (!mbar_wait(q_full, 0, s_abort, p.status)) {
-                ok = false;
-                break;
-              }
-              q_ready = true;
-            }
+          if (j < n[x]) {
+            // S_x = Q_x K_x(j)^T into the same TMEM columns
             if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t k_base = smem_u32(sRing + stage * TILE_BYTES);
-            const uint32_t qx = q_base + x * TILE_BYTES;
+            const uint64_t kd = k_desc0 + ((stage * TILE_BYTES) >> 4);
 #pragma unroll
             for (int c = 0; c < NCHUNK; ++c)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = sdesc_kmajor_sw128(qx + c * CHUNK_BYTES + kk * 32);
-                const uint64_t bd = sdesc_kmajor_sw128(k_base + c * CHUNK_BYTES + kk * 32);
-                mma_bf16_ss(tm_s(x), a, bd, IDESC_S, (c | kk) != 0);
+                const uint32_t off = (c * CHUNK_BYTES + kk * 32) >> 4;
+                mma_bf16_ss(tm_s(x), q_desc[x] + off, kd + off, IDESC_S, (c | kk) != 0);
               }
             mma_commit(&kv_empty[stage]);
             mma_commit(&s_full[x]);
@@ -278,13 +342,8 @@ __global__ void __launch_bounds__(384, 1)
               stage = 0;
               phase ^= 1;
             }
-            ++ntile[x];
-            pend[x] = true;
-            J[x] = cur[x].next(nullptr);
-            any = true;
           }
         }
-        if (!any) break;
       }
       mma_commit(drain);
       mbar_wait_drain(drain, 0);
@@ -349,9 +408,22 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) lsum[c] = fmul2(lsum[c], a2);
       }
+      if (rescale) {
+        // O_x is final for the previous tile (S_x(t) completing implies it). It is rescaled
+        // before any P of this tile is published, since the PV product starts on the first half.
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(o_cols + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tmem_st32(o_cols + c * 32, o);
+        }
+      }
       // pass 2: P = 2^(u*scale_log2 - m) in bf16, written over S. Keys 0..63 are re-read and
-      // packed into columns 0..31 before keys 64..127 are re-read: the packed P of keys 64..127
-      // lands in columns 32..63, whose logits (keys 32..63) are consumed by then.
+      // packed into columns 0..31 and published (p_half) before keys 64..127 are re-read: their
+      // packed P lands in columns 32..63, whose logits (keys 32..63) are consumed by then.
       const uint64_t negm = f2_pack(-m_run, -m_run);
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
@@ -374,22 +446,10 @@ __global__ void __launch_bounds__(384, 1)
           pk[q] = pack_bf16x2(p0, p1);
         }
         tmem_st32(s_cols + h * 32, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(h == 0 ? &p_half[x] : &p_full[x]);
       }
-      if (rescale) {
-        // O_x is final for the previous tile: S_x(t) completing implies it
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_cols + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(o_cols + c * 32, o);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[x]);
     }
     if (valid[x]) {
       __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh[x]) * p.L + I * 128 + r) * D;
@@ -434,7 +494,7 @@ static cudaError_t launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk,
                                  cudaStream_t stream) {
   constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
   constexpr int NSTAGE = (D == 128) ? 5 : 10;
-  const size_t smem = 1024 + TILE * (2 + NSTAGE) + (1 + 2 * NSTAGE + 7) * 8 + 16;
+  const size_t smem = 1024 + TILE * (2 + NSTAGE) + (2 * NSTAGE + 10) * 8 + 16;
   auto kern = bs_attn_fwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -472,6 +532,7 @@ cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, 
   ap.nb = g.nb;
   ap.batch = g.b;
   ap.n_pairs = g.b * ((g.hq + 1) / 2);
+  ap.chunk = (g.g + 1) / 2;
   ap.tri = g.tri;
   ap.scale_log2 = g.scale * 1.4426950408889634f;
   ap.kept_idx = kept_idx;
