@@ -3,8 +3,8 @@
 // digest; online softmax as in FlashAttention / FlashAttention-2), GQA head mapping.
 //
 // One CTA runs two work items side by side: query block I of heads 2c and 2c+1 (of one batch
-// row), each with its own kept list. Grid order is by KV-head chunk, then longest-first (I
-// descending) within the chunk (see attn_item). Roles:
+// row), each with its own kept list. Grid order is longest-first (I descending), by KV-head
+// chunk when K and V exceed L2 (see attn_item). Roles:
 //   warp 0       TMA producer: both Q tiles once, then per step j the tiles V_A(j-1), K_A(j),
 //                V_B(j-1), K_B(j) through a ring of 128-row tiles, in the order the MMA warp
 //                consumes them;
@@ -35,7 +35,7 @@ namespace rra {
 struct AttnParams {
   int hq, hkv, g, L, nb, batch;
   int n_pairs;       // batch * ceil(hq / 2)
-  int chunk;         // head pairs per KV-head chunk of the launch order (ceil(g / 2))
+  int chunk;         // head pairs per chunk of the launch order (ceil(g / 2) or all)
   int64_t tri;
   float scale_log2;
   const int32_t *kept_idx;
@@ -105,10 +105,11 @@ __device__ int count_valid_warp(const AttnParams &p, int bh, int I, bool valid, 
   return n;
 }
 
-// Launch order: per batch row, chunks of `chunk` head pairs (the query heads of about one KV
-// head), each chunk's block rows longest first (I descending), the chunk's pairs innermost. The
-// CTAs resident at one time then read the K/V tiles of one or two KV heads, which fit in L2 even
-// at long lengths, so a tile kept by several rows or heads is fetched from DRAM about once.
+// Launch order: per batch row, chunks of `chunk` head pairs, each chunk's block rows longest
+// first (I descending), the chunk's pairs innermost. With one chunk per batch row this is plain
+// longest-first. With chunks of the query heads of one KV head, the CTAs resident at one time
+// read the K/V tiles of one or two KV heads, which fit in L2 even at long lengths, so a tile kept
+// by several rows or heads is fetched from DRAM about once.
 __device__ __forceinline__ void attn_item(const AttnParams &p, int64_t idx, int &b, int &c,
                                           int &level) {
   const int hp = (p.hq + 1) >> 1;
@@ -503,6 +504,20 @@ static cudaError_t launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk,
   return cudaGetLastError();
 }
 
+// L2 size of the current device (queried once per device)
+static int64_t l2_bytes() {
+  static int64_t cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 128ll << 20;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrL2CacheSize, dev) != cudaSuccess || v <= 0)
+      v = 128 << 20;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
 static bool make_map2d(CUtensorMap *map, const void *base, int64_t rows, int d) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
@@ -532,7 +547,10 @@ cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, 
   ap.nb = g.nb;
   ap.batch = g.b;
   ap.n_pairs = g.b * ((g.hq + 1) / 2);
-  ap.chunk = (g.g + 1) / 2;
+  // KV-head chunks only when K and V of all heads are well beyond L2: then the chunked order
+  // keeps re-read tiles in L2. Below that the plain longest-first order balances the tail better.
+  const int64_t kv_bytes = static_cast<int64_t>(g.b) * g.hkv * g.L * g.d * 2 * 2;
+  ap.chunk = kv_bytes > 2 * l2_bytes() ? (g.g + 1) / 2 : (g.hq + 1) / 2;
   ap.tri = g.tri;
   ap.scale_log2 = g.scale * 1.4426950408889634f;
   ap.kept_idx = kept_idx;
