@@ -334,8 +334,11 @@ __global__ void __launch_bounds__(384, 1)
     int acc = 0;
     uint32_t aph = 0;
     bool dead = false;
-    float *e_base = p.est_e + static_cast<size_t>(blockIdx.x * 128 + r) * p.ntiles * SEG_ROW;
-    float *ref_base = p.est_ref + static_cast<size_t>(blockIdx.x * 128 + r) * p.ntiles * 2;
+    // scratch slot of this CTA, row-contiguous: partial sum (key tile n, segment s, row r) at
+    // e_base[(n * SEG_ROW + s) * 128] and the reference of (n, half) at ref_base[(n * 2 + half)
+    // * 128], so each warp access covers 32 consecutive rows (one 128-byte line)
+    float *e_base = p.est_e + static_cast<size_t>(blockIdx.x) * p.ntiles * SEG_ROW * 128 + r;
+    float *ref_base = p.est_ref + static_cast<size_t>(blockIdx.x) * p.ntiles * 2 * 128 + r;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
       int bh, t;
       est_decode(p, item, bh, t);
@@ -401,17 +404,10 @@ __global__ void __launch_bounds__(384, 1)
           acc = 0;
           aph ^= 1;
         }
-        float *dst = e_base + static_cast<size_t>(n) * SEG_ROW + half * SEG;
-        if constexpr (SEG % 4 == 0) {
+        float *dst = e_base + (static_cast<size_t>(n) * SEG_ROW + half * SEG) * 128;
 #pragma unroll
-          for (int s = 0; s < SEG; s += 4)
-            *reinterpret_cast<float4 *>(dst + s) = make_float4(e[s], e[s + 1], e[s + 2], e[s + 3]);
-        } else {
-#pragma unroll
-          for (int s = 0; s < SEG; s += 2)
-            *reinterpret_cast<float2 *>(dst + s) = make_float2(e[s], e[s + 1]);
-        }
-        ref_base[n * 2 + half] = m_run;
+        for (int s = 0; s < SEG; ++s) dst[s * 128] = e[s];
+        ref_base[(n * 2 + half) * 128] = m_run;
       }
       // ---- combine the two half-rows' running max / sum
       sM[half * 128 + r] = m_run;
@@ -442,21 +438,10 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int s = 0; s < SEG; ++s) e[k][s] = 0.f;
           if (n <= t) {
-            fr[k] = ref_base[n * 2 + half];
-            const float *src = e_base + static_cast<size_t>(n) * SEG_ROW + half * SEG;
-            if constexpr (SEG % 4 == 0) {
+            fr[k] = ref_base[(n * 2 + half) * 128];
+            const float *src = e_base + (static_cast<size_t>(n) * SEG_ROW + half * SEG) * 128;
 #pragma unroll
-              for (int s = 0; s < SEG; s += 4) {
-                const float4 v = *reinterpret_cast<const float4 *>(src + s);
-                e[k][s] = v.x; e[k][s + 1] = v.y; e[k][s + 2] = v.z; e[k][s + 3] = v.w;
-              }
-            } else {
-#pragma unroll
-              for (int s = 0; s < SEG; s += 2) {
-                const float2 v = *reinterpret_cast<const float2 *>(src + s);
-                e[k][s] = v.x; e[k][s + 1] = v.y;
-              }
-            }
+            for (int s = 0; s < SEG; ++s) e[k][s] = src[s * 128];
           }
         }
 #pragma unroll
