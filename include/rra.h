@@ -115,13 +115,13 @@ rra_status rra_prefill(const rra_params *p, const void *q, const void *k, const 
 
 /* Step 1 (estimate) for callers that cannot allocate device memory. It has no counterpart in
  * the paper: it is a convenience of this library. Same inputs, output and validation as
- * rra_estimate, but no workspace argument: the scratch lives in a fixed 32 MiB array inside the
+ * rra_estimate, but no workspace argument: the scratch lives in a fixed 48 MiB array inside the
  * library's device image, which every device that loads the library keeps until the process
  * exits. Meant for callers whose device memory is owned by a pool that forbids new
  * allocations, or that must avoid cudaMalloc / cudaFree because those calls can synchronise the
- * device. Problems whose rra_workspace_bytes exceeds 32 MiB return RRA_ERR_WORKSPACE before
+ * device. Problems whose rra_workspace_bytes exceeds 48 MiB return RRA_ERR_WORKSPACE before
  * anything is enqueued (on a 148-SM B200: a 32-query-head, 8-KV-head, d = 128 layer at S = 8 fits
- * up to 16K tokens). All
+ * up to 23K tokens). All
  * calls share the one array: calls whose kernels may overlap on the GPU (other streams, other
  * threads) race, so serialise them. The first call on each device looks up the array's device
  * address; make it before any stream capture begins. Allocates nothing. */

@@ -19,9 +19,10 @@
 // Qhat . Kbar_hi + Qhat . Kbar_lo (bf16 operands, fp32 accumulation, ~16-bit Kbar), and eight
 // epilogue warps (two per TMEM lane quadrant, one per 64-column half) take the online causal
 // softmax. Because a row's normaliser is known only after its last tile, each thread writes its
-// per-(row, key block) partial sums with the running maximum they were taken against into a
-// per-CTA scratch slot (L2-resident), then rescales them once the row is complete and reduces
-// the m sampled rows of each block row with warp shuffles.
+// per-(row, key block) partial sums with the running maximum they were taken against into the
+// CTA's scratch slot. Four more warps then rescale them once the rows are complete and reduce
+// the m sampled rows of each block row with warp shuffles, while the epilogue warps go on to the
+// next item: the slot holds two buffers, used by alternate items.
 #include <math.h>
 
 #include "common.cuh"
@@ -97,7 +98,7 @@ __device__ __forceinline__ void est_decode(const EstParams &p, int item, int &bh
 // RR: tm_q = 3-D view of Q (box at in-stride offset o_h), tm_khi / tm_klo = pooled keys.
 // XA: tm_q = the same 3-D view of Q, tm_khi = 3-D view of K (box at in-stride offset S-1-t).
 template <int D, int M, bool XA>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     rr_estimate_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_khi,
                        const __grid_constant__ CUtensorMap tm_klo, const EstParams p) {
@@ -124,9 +125,12 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t *acc_full = kv_empty + NSTAGE;         // [2]
   uint64_t *acc_empty = acc_full + 2;             // [2]
   uint64_t *drain = acc_empty + 2;
-  float *sM = reinterpret_cast<float *>(drain + 2);   // [2][128]
-  float *sL = sM + 256;                               // [2][128]
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sL + 256);
+  uint64_t *fp_full = drain + 2;                  // [2] scratch buffer b holds a complete item
+  uint64_t *fp_empty = fp_full + 2;               // [2] scratch buffer b has been reduced
+  float *sM = reinterpret_cast<float *>(fp_empty + 2);   // [2][128]
+  float *sL = sM + 256;                                  // [2][128]
+  float *sRow = sL + 256;     // [2 buffers][2][128]: row max and 1 / row sum of buffer b's item
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sRow + 512);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -144,6 +148,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
       mbar_init(&acc_empty[a], 256);
+      mbar_init(&fp_full[a], 256);
+      mbar_init(&fp_empty[a], 128);
     }
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -325,7 +331,7 @@ __global__ void __launch_bounds__(384, 1)
       mma_commit(drain);   // every MMA issued by this thread completes before teardown
       mbar_wait_drain(drain, 0);
     }
-  } else if (warp >= 4) {
+  } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ softmax / mass epilogue
     const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
     const int half = (warp - 4) >> 2;     // accumulator columns 64*half .. 64*half+63
@@ -334,12 +340,19 @@ __global__ void __launch_bounds__(384, 1)
     int acc = 0;
     uint32_t aph = 0;
     bool dead = false;
-    // scratch slot of this CTA, row-contiguous: partial sum (key tile n, segment s, row r) at
-    // e_base[(n * SEG_ROW + s) * 128] and the reference of (n, half) at ref_base[(n * 2 + half)
-    // * 128], so each warp access covers 32 consecutive rows (one 128-byte line)
-    float *e_base = p.est_e + static_cast<size_t>(blockIdx.x) * p.ntiles * SEG_ROW * 128 + r;
-    float *ref_base = p.est_ref + static_cast<size_t>(blockIdx.x) * p.ntiles * 2 * 128 + r;
-    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x) {
+    int kit = 0;   // this CTA's item ordinal; its scratch buffer is kit & 1
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++kit) {
+      const int buf = kit & 1;
+      // scratch buffer, row-contiguous: partial sum (key tile n, segment s, row r) at
+      // e_base[(n * SEG_ROW + s) * 128] and the reference of (n, half) at
+      // ref_base[(n * 2 + half) * 128], so each warp access covers one 128-byte line
+      float *e_base = p.est_e + (static_cast<size_t>(blockIdx.x) * 2 + buf) * p.ntiles * SEG_ROW *
+                                    128 + r;
+      float *ref_base =
+          p.est_ref + (static_cast<size_t>(blockIdx.x) * 2 + buf) * p.ntiles * 2 * 128 + r;
+      // the buffer's previous item (kit - 2) must have been reduced
+      if (!dead && kit >= 2)
+        dead = !mbar_wait_warp(&fp_empty[buf], ((kit >> 1) - 1) & 1, s_abort, p.status);
       int bh, t;
       est_decode(p, item, bh, t);
       const int i = t * 128 + r;          // sampled query (stride) index of this row
@@ -420,38 +433,69 @@ __global__ void __launch_bounds__(384, 1)
       if (m1 > NEG_INF) ltot += sL[128 + r] * fast_exp2(m1 - mx);
       named_bar_sync(1, 256);
       const float inv = (row_ok && ltot > 0.f) ? 1.f / ltot : 0.f;
-      // ---- rescale the partial sums and reduce the M sampled rows of each block row
+      if (half == 0) {
+        sRow[buf * 256 + r] = mx;
+        sRow[buf * 256 + 128 + r] = inv;
+      }
+      // publishes this thread's partial sums and, for half 0, the row's max and 1 / sum
+      mbar_arrive(&fp_full[buf]);
+    }
+    tc_fence_before();
+  } else if (warp >= 12) {
+    // ------------------------------------------------------------ partial-sum reduction
+    // One thread per row of buffer kit & 1's item: rescale the row's partial sums by
+    // 2^(ref - max) / sum and reduce the M sampled rows of each block row (M consecutive lanes).
+    const int r = (warp - 12) * 32 + lane;
+    const float NEG_INF = -INFINITY;
+    int kit = 0;
+    for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++kit) {
+      const int buf = kit & 1;
+      if (!mbar_wait_warp(&fp_full[buf], (kit >> 1) & 1, s_abort, p.status)) break;
+      const float *e_base = p.est_e + (static_cast<size_t>(blockIdx.x) * 2 + buf) * p.ntiles *
+                                          SEG_ROW * 128 + r;
+      const float *ref_base =
+          p.est_ref + (static_cast<size_t>(blockIdx.x) * 2 + buf) * p.ntiles * 2 * 128 + r;
+      int bh, t;
+      est_decode(p, item, bh, t);
+      const int i = t * 128 + r;
+      const bool row_ok = i < p.ns;
+      const float mx = sRow[buf * 256 + r];
+      const float inv = sRow[buf * 256 + 128 + r];
       const int I = i / M;
       float *mass_row = p.mass + static_cast<int64_t>(bh) * p.tri +
                         static_cast<int64_t>(I) * (I + 1) / 2;
       const bool writer = row_ok && ((lane % M) == 0);
       // PF key tiles per batch: all their loads are issued before any is used, so the loop
-      // pays one L2 round trip per batch instead of one per tile
-      constexpr int PF = (SEG >= 32) ? 1 : 32 / SEG;
+      // pays one L2 / DRAM round trip per batch instead of one per tile
+      constexpr int PF = (SEG_ROW >= 32) ? 1 : 32 / SEG_ROW;
       for (int n0 = 0; n0 <= t; n0 += PF) {
-        float fr[PF];
-        float e[PF][SEG];
+        float fr[PF][2];
+        float e[PF][SEG_ROW];
 #pragma unroll
         for (int k = 0; k < PF; ++k) {
           const int n = n0 + k;
-          fr[k] = NEG_INF;
+          fr[k][0] = fr[k][1] = NEG_INF;
 #pragma unroll
-          for (int s = 0; s < SEG; ++s) e[k][s] = 0.f;
+          for (int s = 0; s < SEG_ROW; ++s) e[k][s] = 0.f;
           if (n <= t) {
-            fr[k] = ref_base[(n * 2 + half) * 128];
-            const float *src = e_base + (static_cast<size_t>(n) * SEG_ROW + half * SEG) * 128;
+            fr[k][0] = ref_base[(n * 2) * 128];
+            fr[k][1] = ref_base[(n * 2 + 1) * 128];
+            const float *src = e_base + static_cast<size_t>(n) * SEG_ROW * 128;
 #pragma unroll
-            for (int s = 0; s < SEG; ++s) e[k][s] = src[s * 128];
+            for (int s = 0; s < SEG_ROW; ++s) e[k][s] = src[s * 128];
           }
         }
 #pragma unroll
         for (int k = 0; k < PF; ++k) {
           const int n = n0 + k;
-          const float f = (inv > 0.f && fr[k] > NEG_INF) ? fast_exp2(fr[k] - mx) * inv : 0.f;
-          const int jb0 = (n * 128 + half * 64) / M;
+          float f[2];
 #pragma unroll
-          for (int s = 0; s < SEG; ++s) {
-            float v = e[k][s] * f;
+          for (int hh = 0; hh < 2; ++hh)
+            f[hh] = (inv > 0.f && fr[k][hh] > NEG_INF) ? fast_exp2(fr[k][hh] - mx) * inv : 0.f;
+          const int jb0 = (n * 128) / M;
+#pragma unroll
+          for (int s = 0; s < SEG_ROW; ++s) {
+            float v = e[k][s] * f[s / SEG];
 #pragma unroll
             for (int off = M / 2; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
             const int J = jb0 + s;
@@ -459,6 +503,8 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
+      // every load of this buffer has returned (its values were used above)
+      mbar_arrive(&fp_empty[buf]);
     }
     tc_fence_before();
   }
@@ -509,13 +555,13 @@ static cudaError_t launch_est_t(const CUtensorMap &mq, const CUtensorMap &mhi,
                                 cudaStream_t stream) {
   constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
   constexpr int NSTAGE = XA ? 3 : 2;
-  const size_t smem = 1024 + TILE * ((XA ? 0 : 1) + 2 * NSTAGE) + (2 + 2 * NSTAGE + 6) * 8 +
-                      512 * 4 + 16;
+  const size_t smem = 1024 + TILE * ((XA ? 0 : 1) + 2 * NSTAGE) + (2 + 2 * NSTAGE + 10) * 8 +
+                      1024 * 4 + 16;
   auto kern = rr_estimate_kernel<D, M, XA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<slots, 384, smem, stream>>>(mq, mhi, mlo, ep);
+  kern<<<slots, 512, smem, stream>>>(mq, mhi, mlo, ep);
   return cudaGetLastError();
 }
 

@@ -25,10 +25,11 @@ WorkspaceLayout workspace_layout(const Geometry &g, int num_sms) {
   if (items < slots) slots = static_cast<int>(items < 1 ? 1 : items);
   w.est_slots = slots;
   const int segs = g.m > 0 ? 128 / g.m : 0;
+  // two scratch buffers per slot: one item is reduced while the next is computed
   w.est_e = align_up(off, 256);
-  off = w.est_e + static_cast<size_t>(slots) * 128 * g.ntiles * segs * 4;
+  off = w.est_e + static_cast<size_t>(slots) * 2 * 128 * g.ntiles * segs * 4;
   w.est_ref = align_up(off, 256);
-  off = w.est_ref + static_cast<size_t>(slots) * 128 * g.ntiles * 2 * 4;
+  off = w.est_ref + static_cast<size_t>(slots) * 2 * 128 * g.ntiles * 2 * 4;
   w.mass = align_up(off, 256);
   off = w.mass + static_cast<size_t>(g.b) * g.hq * g.tri * 4;
   w.total = align_up(off, 256);

@@ -9,7 +9,7 @@
 // a device and stays allocated on every device that uses the library until the process exits.
 //
 // Costs and limits:
-//   - kStaticScratchBytes (32 MiB) bounds the problems it accepts; larger ones are refused with
+//   - kStaticScratchBytes (48 MiB) bounds the problems it accepts; larger ones are refused with
 //     RRA_ERR_WORKSPACE before anything is enqueued.
 //   - All calls share the one array, so two calls whose kernels overlap on a GPU (different
 //     streams, or different host threads) race and corrupt each other's results. Serialise
@@ -25,7 +25,7 @@
 
 namespace {
 
-constexpr size_t kStaticScratchBytes = static_cast<size_t>(32) << 20;
+constexpr size_t kStaticScratchBytes = static_cast<size_t>(48) << 20;
 constexpr int kMaxDevices = 64;
 
 // The scratch itself. Host code must not pass `g_rra_static_scratch` to a kernel: on the host

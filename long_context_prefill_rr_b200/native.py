@@ -163,7 +163,7 @@ def estimate_xattn(p: RraParams, q, k, mass, ws, stream=None):
 
 def estimate_static_scratch(p: RraParams, q, k, mass, stream=None):
     """rra_estimate without a workspace, for callers that cannot allocate device memory: the
-    library's fixed 32 MiB device array serves as scratch (problems that need more are
+    library's fixed 48 MiB device array serves as scratch (problems that need more are
     refused; calls that overlap on the GPU race on the shared array)."""
     import torch
     sh = shapes(p)
