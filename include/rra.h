@@ -113,6 +113,29 @@ rra_status rra_prefill(const rra_params *p, const void *q, const void *k, const 
                        void *out, float *mass, int32_t *kept_idx, int32_t *kept_cnt,
                        void *workspace, size_t workspace_bytes, rra_stream_t stream);
 
+/* Steps 1-3 on HOST inputs and output, with the copies overlapped with the compute. It has no
+ * counterpart in the paper: it is a convenience of this library. q_host, k_host, v_host and
+ * out_host are host buffers in the layouts of rra_prefill; pinned (page-locked) memory lets the
+ * copies run asynchronously. q_dev, k_dev, v_dev, out_dev are device staging buffers of the same
+ * sizes, kept_idx / kept_cnt device outputs as in rra_prefill; the masses stay in the workspace,
+ * which must hold rra_workspace_bytes(p).
+ * The problem is cut into up to 8 chunks: groups of KV heads (with their query heads) when
+ * batch == 1, else groups of batch rows. Each chunk is an independent sub-problem, because every
+ * step is per (batch row, head); a chunk of heads runs with the round-robin shift advanced by its
+ * first query head, so every head samples the offset it would sample in the whole problem, and
+ * the results equal rra_prefill's. Chunk c's host-to-device copies run on an internal stream,
+ * its estimate, select and attention on `stream` once they have landed, and its output copy on
+ * a second internal stream, so chunk c+1's inputs and chunk c-1's output cross PCIe while chunk
+ * c computes. Each copy is one cudaMemcpyAsync. The call is asynchronous: `stream` completes
+ * after the last output copy, and the staging buffers are used only after the work already on
+ * `stream`. The internal streams and events are created on the first call on each device (make
+ * it before any stream capture) and kept until exit; calls on one device must not overlap.
+ * Errors as for rra_prefill. */
+rra_status rra_prefill_host(const rra_params *p, const void *q_host, const void *k_host,
+                            const void *v_host, void *out_host, void *q_dev, void *k_dev,
+                            void *v_dev, void *out_dev, int32_t *kept_idx, int32_t *kept_cnt,
+                            void *workspace, size_t workspace_bytes, rra_stream_t stream);
+
 /* Step 1 (estimate) for callers that cannot allocate device memory. It has no counterpart in
  * the paper: it is a convenience of this library. Same inputs, output and validation as
  * rra_estimate, but no workspace argument: the scratch lives in a fixed 48 MiB array inside the

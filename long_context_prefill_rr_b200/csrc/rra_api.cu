@@ -1,6 +1,8 @@
 // C ABI of the RRAttention prefill hot path (declared in include/rra.h): argument validation,
 // workspace carve-up and kernel launches. No memory is allocated here.
 #include <math.h>
+
+#include <algorithm>
 #include <mutex>
 
 #include "rra.h"
@@ -131,6 +133,51 @@ rra_status run_estimate(const Geometry &g, const void *q, const void *k, float *
   return cuda_status(e);
 }
 
+rra_status run_prefill(const Geometry &g, const void *q, const void *k, const void *v, void *out,
+                       float *mass, int32_t *kept_idx, int32_t *kept_cnt, void *workspace,
+                       const WorkspaceLayout &w, int sms, cudaStream_t st) {
+  float *m = mass ? mass : ws_at<float>(workspace, w.mass);
+  rra_status s = run_estimate(g, q, k, m, workspace, w, sms, st);
+  if (s != RRA_OK) return s;
+  if (rra::launch_topt_select(g, m, kept_idx, kept_cnt, sms, st) != cudaSuccess)
+    return RRA_ERR_CUDA;
+  return cuda_status(rra::launch_sparse_attn(g, q, k, v, kept_idx, kept_cnt, out,
+                                             status_word(workspace, w), st));
+}
+
+// Streams and events of rra_prefill_host, created once per device.
+constexpr int kMaxHostChunks = 8;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_done[kMaxHostChunks] = {};
+  cudaEvent_t step_done[kMaxHostChunks] = {};
+  bool ready = false;
+};
+
+HostPipe *host_pipe() {
+  static std::mutex mu;
+  static HostPipe pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  HostPipe &hp = pipes[dev];
+  if (!hp.ready) {
+    const unsigned ef = cudaEventDisableTiming;
+    if (cudaStreamCreateWithFlags(&hp.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&hp.out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.start, ef) != cudaSuccess ||
+        cudaEventCreateWithFlags(&hp.end, ef) != cudaSuccess)
+      return nullptr;
+    for (int c = 0; c < kMaxHostChunks; ++c)
+      if (cudaEventCreateWithFlags(&hp.in_done[c], ef) != cudaSuccess ||
+          cudaEventCreateWithFlags(&hp.step_done[c], ef) != cudaSuccess)
+        return nullptr;
+    hp.ready = true;
+  }
+  return &hp;
+}
+
 }  // namespace
 
 extern "C" {
@@ -216,14 +263,87 @@ rra_status rra_prefill(const rra_params *p, const void *q, const void *k, const 
   if (sms <= 0) return RRA_ERR_CUDA;
   const WorkspaceLayout w = rra::workspace_layout(g, sms);
   if (workspace_bytes < w.total) return RRA_ERR_WORKSPACE;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  float *m = mass ? mass : ws_at<float>(workspace, w.mass);
-  s = run_estimate(g, q, k, m, workspace, w, sms, st);
+  return run_prefill(g, q, k, v, out, mass, kept_idx, kept_cnt, workspace, w, sms,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+rra_status rra_prefill_host(const rra_params *p, const void *q_host, const void *k_host,
+                            const void *v_host, void *out_host, void *q_dev, void *k_dev,
+                            void *v_dev, void *out_dev, int32_t *kept_idx, int32_t *kept_cnt,
+                            void *workspace, size_t workspace_bytes, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, kNeedsStride | kNeedsHeadDim, &g);
   if (s != RRA_OK) return s;
-  if (rra::launch_topt_select(g, m, kept_idx, kept_cnt, sms, st) != cudaSuccess)
+  if (empty(g)) return RRA_OK;
+  if (!q_host || !k_host || !v_host || !out_host || !ptr_ok(q_dev) || !ptr_ok(k_dev) ||
+      !ptr_ok(v_dev) || !ptr_ok(out_dev) || !ptr_ok(kept_idx) || !ptr_ok(kept_cnt) ||
+      !ptr_ok(workspace))
+    return RRA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return RRA_ERR_CUDA;
+  if (workspace_bytes < rra::workspace_layout(g, sms).total) return RRA_ERR_WORKSPACE;
+  HostPipe *hp = host_pipe();
+  if (!hp) return RRA_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // chunks: KV-head groups of the one batch row, or batch rows; each chunk is a whole
+  // sub-problem with contiguous inputs, outputs and kept lists
+  const bool by_heads = g.b == 1;
+  const int units = by_heads ? g.hkv : g.b;
+  const int per = (units + kMaxHostChunks - 1) / kMaxHostChunks;
+  const int nch = (units + per - 1) / per;
+  const size_t row_q = static_cast<size_t>(g.L) * g.d * 2;   // bytes of one head's rows
+  const size_t q_unit = by_heads ? row_q * g.g : row_q * g.hq;
+  const size_t kv_unit = by_heads ? row_q : row_q * g.hkv;
+  const int64_t idx_unit = by_heads ? static_cast<int64_t>(g.g) * g.tri
+                                    : static_cast<int64_t>(g.hq) * g.tri;
+  const int64_t cnt_unit = by_heads ? static_cast<int64_t>(g.g) * g.nb
+                                    : static_cast<int64_t>(g.hq) * g.nb;
+  auto at = [](const void *base, size_t off) {
+    return const_cast<uint8_t *>(static_cast<const uint8_t *>(base)) + off;
+  };
+  // the staging buffers may still be in use by earlier work on the caller's stream
+  if (cudaEventRecord(hp->start, st) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
     return RRA_ERR_CUDA;
-  return cuda_status(rra::launch_sparse_attn(g, q, k, v, kept_idx, kept_cnt, out,
-                                             status_word(workspace, w), st));
+  for (int c = 0; c < nch; ++c) {
+    const int u0 = c * per, u1 = std::min(units, u0 + per), nu = u1 - u0;
+    rra_params cp = *p;
+    if (by_heads) {
+      cp.heads_kv = nu;
+      cp.heads_q = nu * g.g;
+      cp.shift = (g.shift + u0 * g.g) % g.S;   // the chunk's heads keep their global offsets
+    } else {
+      cp.batch = nu;
+    }
+    Geometry cg;
+    if (resolve(&cp, kNeedsStride | kNeedsHeadDim, &cg) != RRA_OK) return RRA_ERR_INVALID_ARG;
+    const WorkspaceLayout cw = rra::workspace_layout(cg, sms);
+    const size_t qo = q_unit * u0, kvo = kv_unit * u0;
+    const size_t qb = q_unit * nu, kvb = kv_unit * nu;
+    if (cudaMemcpyAsync(at(q_dev, qo), at(q_host, qo), qb, cudaMemcpyHostToDevice, hp->in) !=
+            cudaSuccess ||
+        cudaMemcpyAsync(at(k_dev, kvo), at(k_host, kvo), kvb, cudaMemcpyHostToDevice,
+                        hp->in) != cudaSuccess ||
+        cudaMemcpyAsync(at(v_dev, kvo), at(v_host, kvo), kvb, cudaMemcpyHostToDevice,
+                        hp->in) != cudaSuccess ||
+        cudaEventRecord(hp->in_done[c], hp->in) != cudaSuccess ||
+        cudaStreamWaitEvent(st, hp->in_done[c], 0) != cudaSuccess)
+      return RRA_ERR_CUDA;
+    s = run_prefill(cg, at(q_dev, qo), at(k_dev, kvo), at(v_dev, kvo), at(out_dev, qo), nullptr,
+                    kept_idx + idx_unit * u0, kept_cnt + cnt_unit * u0, workspace, cw, sms, st);
+    if (s != RRA_OK) return s;
+    if (cudaEventRecord(hp->step_done[c], st) != cudaSuccess ||
+        cudaStreamWaitEvent(hp->out, hp->step_done[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(at(out_host, qo), at(out_dev, qo), qb, cudaMemcpyDeviceToHost,
+                        hp->out) != cudaSuccess)
+      return RRA_ERR_CUDA;
+  }
+  // the call is complete, on the caller's stream, once the last output copy has landed
+  if (cudaEventRecord(hp->end, hp->out) != cudaSuccess ||
+      cudaStreamWaitEvent(st, hp->end, 0) != cudaSuccess)
+    return RRA_ERR_CUDA;
+  return RRA_OK;
 }
 
 rra_status rra_check_device_status(void *workspace, rra_stream_t stream, uint32_t *raw_word) {

@@ -32,6 +32,8 @@ _SIGS = {
     "rra_prefill": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
                                _c.c_void_p]),
+    "rra_prefill_host": (_c.c_int, [_c.c_void_p] + [_c.c_void_p] * 11 + [_c.c_size_t,
+                                                                          _c.c_void_p]),
     "rra_estimate_xattn": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                       _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "rra_estimate_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p,
@@ -219,6 +221,29 @@ def check_device_status(ws, stream=None) -> tuple[int, int]:
     raw = ctypes.c_uint32(0)
     st = load().rra_check_device_status(_ptr(ws), _stream(stream), ctypes.byref(raw))
     return int(st), int(raw.value)
+
+
+def prefill_host(p: RraParams, q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev,
+                 kept_idx, kept_cnt, ws, stream=None):
+    """rra_prefill_host: host (preferably pinned) bf16 q/k/v in, host bf16 out, with device
+    staging buffers of the same shapes; chunked so that copies overlap the compute."""
+    import torch
+    sh = shapes(p)
+    for t, name, shp in ((q_host, "q_host", sh["q"]), (k_host, "k_host", sh["kv"]),
+                         (v_host, "v_host", sh["kv"]), (out_host, "out_host", sh["q"])):
+        if t.device.type != "cpu" or t.dtype != torch.bfloat16 or tuple(t.shape) != shp \
+                or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous CPU bf16 tensor of shape {shp}")
+    _expect(q_dev, torch.bfloat16, sh["q"], "q_dev")
+    _expect(k_dev, torch.bfloat16, sh["kv"], "k_dev")
+    _expect(v_dev, torch.bfloat16, sh["kv"], "v_dev")
+    _expect(out_dev, torch.bfloat16, sh["q"], "out_dev")
+    _expect(kept_idx, torch.int32, sh["kept_idx"], "kept_idx")
+    _expect(kept_cnt, torch.int32, sh["kept_cnt"], "kept_cnt")
+    _check(load().rra_prefill_host(_p(p), _ptr(q_host), _ptr(k_host), _ptr(v_host),
+                                   _ptr(out_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev),
+                                   _ptr(out_dev), _ptr(kept_idx), _ptr(kept_cnt), _ptr(ws),
+                                   ws.numel(), _stream(stream)), "rra_prefill_host")
 
 
 def new_workspace(p: RraParams, device=None):

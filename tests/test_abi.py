@@ -29,7 +29,8 @@ def lib():
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
         "rra_workspace_bytes", "rra_estimate", "rra_select", "rra_sparse_attn", "rra_prefill",
-        "rra_estimate_static_scratch", "rra_estimate_xattn", "rra_check_device_status",
+        "rra_estimate_static_scratch", "rra_estimate_xattn", "rra_prefill_host",
+        "rra_check_device_status",
         "rra_status_string", "rra_version"])
 
 
@@ -80,6 +81,12 @@ def test_pointer_checks(lib):
     assert lib.rra_select(ctypes.byref(p), None, ctypes.c_void_p(16), ctypes.c_void_p(16),
                           None) == 1
     assert lib.rra_check_device_status(None, None, None) == 1
+    # host entry: a missing host buffer or a misaligned staging buffer is refused up front
+    ok, bad = ctypes.c_void_p(16), ctypes.c_void_p(8)
+    assert lib.rra_prefill_host(ctypes.byref(p), None, ok, ok, ok, ok, ok, ok, ok, ok, ok, ok,
+                                1 << 30, None) == 1
+    assert lib.rra_prefill_host(ctypes.byref(p), ok, ok, ok, ok, bad, ok, ok, ok, ok, ok, ok,
+                                1 << 30, None) == 1
 
 
 def test_empty_problem_is_a_noop(lib):
