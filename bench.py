@@ -384,8 +384,8 @@ def run_gpu(args, w):
             "e2e": {"value": e2e_ms if sharded else e2e_ms / ws_n, "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d_all), "d2h_bytes_per_step": int(d2h_all)},
             "gpu_launches": 4 * args.steps,
-            "e2e_api": "rra_prefill_host (pinned host buffers; copies overlapped per KV-head "
-                       "chunk)",
+            "e2e_api": "rra_prefill_host (pinned host buffers; copies overlapped with the "
+                       "compute, chunk by chunk)",
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

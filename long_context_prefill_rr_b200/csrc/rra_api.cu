@@ -146,7 +146,7 @@ rra_status run_prefill(const Geometry &g, const void *q, const void *k, const vo
 }
 
 // Streams and events of rra_prefill_host, created once per device.
-constexpr int kMaxHostChunks = 8;
+constexpr int kMaxHostChunks = 16;
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, end = nullptr;
@@ -285,19 +285,37 @@ rra_status rra_prefill_host(const rra_params *p, const void *q_host, const void 
   HostPipe *hp = host_pipe();
   if (!hp) return RRA_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // chunks: KV-head groups of the one batch row, or batch rows; each chunk is a whole
-  // sub-problem with contiguous inputs, outputs and kept lists
-  const bool by_heads = g.b == 1;
-  const int units = by_heads ? g.hkv : g.b;
-  const int per = (units + kMaxHostChunks - 1) / kMaxHostChunks;
-  const int nch = (units + per - 1) / per;
+  // Chunks, each a whole sub-problem with contiguous inputs, outputs and kept lists. At batch 1:
+  // groups of query heads within one KV head (a divisor gq of the GQA group, as small as keeps
+  // the chunk count within kMaxHostChunks; a KV head's K and V travel with its first group), or
+  // whole KV heads when there are more KV heads than chunks. Otherwise: groups of batch rows.
+  struct Chunk {
+    int b0, nb, h0, nh, kv0, nkv;
+    bool copy_kv;
+  };
+  Chunk ch[kMaxHostChunks];
+  int nch = 0;
+  if (g.b == 1) {
+    if (g.hkv <= kMaxHostChunks) {
+      int gq = g.g;
+      for (int d = g.g - 1; d >= 1; --d)
+        if (g.g % d == 0 && g.hkv * (g.g / d) <= kMaxHostChunks) gq = d;
+      for (int kv = 0; kv < g.hkv; ++kv)
+        for (int j = 0; j < g.g / gq; ++j)
+          ch[nch++] = {0, 1, kv * g.g + j * gq, gq, kv, 1, j == 0};
+    } else {
+      const int per = (g.hkv + kMaxHostChunks - 1) / kMaxHostChunks;
+      for (int kv = 0; kv < g.hkv; kv += per) {
+        const int n = std::min(per, g.hkv - kv);
+        ch[nch++] = {0, 1, kv * g.g, n * g.g, kv, n, true};
+      }
+    }
+  } else {
+    const int per = (g.b + kMaxHostChunks - 1) / kMaxHostChunks;
+    for (int b = 0; b < g.b; b += per)
+      ch[nch++] = {b, std::min(per, g.b - b), 0, g.hq, 0, g.hkv, true};
+  }
   const size_t row_q = static_cast<size_t>(g.L) * g.d * 2;   // bytes of one head's rows
-  const size_t q_unit = by_heads ? row_q * g.g : row_q * g.hq;
-  const size_t kv_unit = by_heads ? row_q : row_q * g.hkv;
-  const int64_t idx_unit = by_heads ? static_cast<int64_t>(g.g) * g.tri
-                                    : static_cast<int64_t>(g.hq) * g.tri;
-  const int64_t cnt_unit = by_heads ? static_cast<int64_t>(g.g) * g.nb
-                                    : static_cast<int64_t>(g.hq) * g.nb;
   auto at = [](const void *base, size_t off) {
     return const_cast<uint8_t *>(static_cast<const uint8_t *>(base)) + off;
   };
@@ -307,31 +325,32 @@ rra_status rra_prefill_host(const rra_params *p, const void *q_host, const void 
       cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
     return RRA_ERR_CUDA;
   for (int c = 0; c < nch; ++c) {
-    const int u0 = c * per, u1 = std::min(units, u0 + per), nu = u1 - u0;
+    const Chunk &k = ch[c];
     rra_params cp = *p;
-    if (by_heads) {
-      cp.heads_kv = nu;
-      cp.heads_q = nu * g.g;
-      cp.shift = (g.shift + u0 * g.g) % g.S;   // the chunk's heads keep their global offsets
-    } else {
-      cp.batch = nu;
-    }
+    cp.batch = k.nb;
+    cp.heads_q = k.nh;
+    cp.heads_kv = k.nkv;
+    cp.shift = (g.shift + k.h0) % g.S;   // the chunk's heads keep their global offsets
     Geometry cg;
     if (resolve(&cp, kNeedsStride | kNeedsHeadDim, &cg) != RRA_OK) return RRA_ERR_INVALID_ARG;
     const WorkspaceLayout cw = rra::workspace_layout(cg, sms);
-    const size_t qo = q_unit * u0, kvo = kv_unit * u0;
-    const size_t qb = q_unit * nu, kvb = kv_unit * nu;
+    // offsets within the [b, H, ...] arrays: batch rows first, then heads
+    const size_t qo = row_q * (static_cast<size_t>(k.b0) * g.hq + k.h0);
+    const size_t qb = row_q * static_cast<size_t>(k.nb) * k.nh;
+    const size_t kvo = row_q * (static_cast<size_t>(k.b0) * g.hkv + k.kv0);
+    const size_t kvb = row_q * static_cast<size_t>(k.nb) * k.nkv;
+    const int64_t lo = static_cast<int64_t>(k.b0) * g.hq + k.h0;   // first (batch, head) row
     if (cudaMemcpyAsync(at(q_dev, qo), at(q_host, qo), qb, cudaMemcpyHostToDevice, hp->in) !=
             cudaSuccess ||
-        cudaMemcpyAsync(at(k_dev, kvo), at(k_host, kvo), kvb, cudaMemcpyHostToDevice,
-                        hp->in) != cudaSuccess ||
-        cudaMemcpyAsync(at(v_dev, kvo), at(v_host, kvo), kvb, cudaMemcpyHostToDevice,
-                        hp->in) != cudaSuccess ||
+        (k.copy_kv && (cudaMemcpyAsync(at(k_dev, kvo), at(k_host, kvo), kvb,
+                                       cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+                       cudaMemcpyAsync(at(v_dev, kvo), at(v_host, kvo), kvb,
+                                       cudaMemcpyHostToDevice, hp->in) != cudaSuccess)) ||
         cudaEventRecord(hp->in_done[c], hp->in) != cudaSuccess ||
         cudaStreamWaitEvent(st, hp->in_done[c], 0) != cudaSuccess)
       return RRA_ERR_CUDA;
     s = run_prefill(cg, at(q_dev, qo), at(k_dev, kvo), at(v_dev, kvo), at(out_dev, qo), nullptr,
-                    kept_idx + idx_unit * u0, kept_cnt + cnt_unit * u0, workspace, cw, sms, st);
+                    kept_idx + lo * g.tri, kept_cnt + lo * g.nb, workspace, cw, sms, st);
     if (s != RRA_OK) return s;
     if (cudaEventRecord(hp->step_done[c], st) != cudaSuccess ||
         cudaStreamWaitEvent(hp->out, hp->step_done[c], 0) != cudaSuccess ||

@@ -1,7 +1,8 @@
 """rra_prefill_host: host buffers in and out, chunked so that the copies overlap the compute.
-Its kept lists and output equal rra_prefill's on the same inputs, bit for bit: the chunks (KV-head
-groups at batch 1, batch rows otherwise) are independent sub-problems, and a chunk of heads runs
-with the round-robin shift advanced by its first head."""
+Its kept lists and output equal rra_prefill's on the same inputs, bit for bit. The chunks are
+independent sub-problems: query-head groups within a KV head, whole KV heads when there are more
+than 16, or batch rows. A chunk of heads runs with the round-robin shift advanced by its first
+head. The cases cover each kind of chunk."""
 import numpy as np
 import pytest
 import torch
@@ -17,6 +18,7 @@ CASES = {
     "llama8k": (wl.WORKLOADS["llama8k"], 1),
     "tiny_batch3": (wl.WORKLOADS["tiny"].with_(heads_kv=2, shift=3), 3),
     "video_short": (wl.WORKLOADS["video64k"].with_(seqlen=4096), 1),
+    "tiny_mha32": (wl.WORKLOADS["tiny"].with_(heads_q=32, heads_kv=32, shift=1), 1),
 }
 
 
