@@ -134,22 +134,6 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
       : "memory");
 }
 
-// Prefetch a tile into L2 (no shared memory, no completion tracking).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int32_t c0, int32_t c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int32_t c0, int32_t c1,
-                                                   int32_t c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1), "r"(c2)
-               : "memory");
-}
-
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -258,16 +242,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -275,16 +249,6 @@ __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
-// Register re-balancing between warpgroups (all four warps of a warpgroup execute the same
-// instruction). The block keeps the registers it was launched with; the shares must add up.
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
 
 // ---------------------------------------------------------------- math
 // 2^x on the special-function unit (PTX ex2.approx.ftz.f32: relative error ~2^-22).
@@ -332,35 +296,6 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-// 2^x for two values on the FMA/ALU pipes instead of the special-function unit. Valid for
-// x in [-125, 128): x = n + f with n = round(x) (magic-number addition) and |f| <= 1/2; 2^f
-// from a degree-3 polynomial whose coefficients were fitted for this library to minimise the
-// relative error on [-1/2, 1/2] (Lawson's iteratively reweighted least squares on Chebyshev
-// nodes; max relative error 7.5e-5 in fp32); 2^n is added into the exponent field. The bits of
-// r = x + 1.5 * 2^23 are 0x4B400000 + n, and (0x4B400000 << 23) vanishes mod 2^32, so the
-// scaled result is bits(p) + (bits(r) << 23). Callers clamp x >= -125.
-__device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t xy) {
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-  const uint64_t negmagic = f2_pack(-12582912.f, -12582912.f);
-  const uint64_t minus1 = f2_pack(-1.f, -1.f);
-  const uint64_t r = fadd2(xy, magic);
-  const uint64_t n = fadd2(r, negmagic);
-  const uint64_t f = ffma2(n, minus1, xy);
-  uint64_t q = ffma2(f2_pack(0.0551716648f, 0.0551716648f), f, f2_pack(0.2426111251f, 0.2426111251f));
-  q = ffma2(q, f, f2_pack(0.6932609677f, 0.6932609677f));
-  q = ffma2(q, f, f2_pack(0.9999280572f, 0.9999280572f));
-  const uint32_t lo = static_cast<uint32_t>(q) + (static_cast<uint32_t>(r) << 23);
-  const uint32_t hi = static_cast<uint32_t>(q >> 32) + (static_cast<uint32_t>(r >> 32) << 23);
-  return (static_cast<uint64_t>(hi) << 32) | lo;
-}
-
-// Two fp32 -> packed bf16x2 without the conversion unit: add half a bf16 ulp to the bits and
-// keep the upper halves (round half away from zero; equals round-to-nearest-even except on
-// exact ties). For finite, non-negative inputs below the bf16 maximum.
-__device__ __forceinline__ uint32_t pack_bf16x2_int(float lo, float hi) {
-  return __byte_perm(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -234,6 +234,22 @@ def test_llama32k_parity(cuda_device, S, tau):
     _sampled_check(w, p, bits, gpu, f"llama32k_S{S}_tau{tau}", n_rows=64, n_attn_rows=16, seed=2)
 
 
+@pytest.mark.parametrize("label,base,over", [
+    # d = 64: the attention's 10-stage ring and the estimate's 64-wide tiles at length
+    ("llama8k_d64", "llama8k", dict(head_dim=64)),
+    # the widest and the narrowest stride: m = 4 and m = 32 sampled rows per block row
+    ("llama16k_s32", "llama32k", dict(seqlen=16384, stride=32)),
+    ("llama16k_s4_shift7", "llama32k", dict(seqlen=16384, stride=4, shift=7)),
+    # two batch rows at length
+    ("llama8k_b2", "llama8k", dict(batch=2)),
+])
+def test_long_variants_parity(cuda_device, label, base, over):
+    w, p = par.workload_params(wl.WORKLOADS[base], **over)
+    bits, dev = _prepare(w)
+    gpu = par.run_prefill(p, *dev)
+    _sampled_check(w, p, bits, gpu, label, n_rows=48, n_attn_rows=12, seed=5)
+
+
 def test_video64k_parity(cuda_device):
     w, p = par.workload_params(wl.WORKLOADS["video64k"])
     bits, dev = _prepare(w)
