@@ -17,8 +17,10 @@
 // sampled queries); the CTA streams the 128-stride key tiles n = 0..t through a 2-stage TMA
 // ring, the MMA warp computes each 128x128 logit tile into one of two TMEM accumulators as
 // Qhat . Kbar_hi + Qhat . Kbar_lo (bf16 operands, fp32 accumulation, ~16-bit Kbar), and eight
-// epilogue warps (two per TMEM lane quadrant, one per 64-column half) take the online causal
-// softmax. Because a row's normaliser is known only after its last tile, each thread writes its
+// epilogue warps take the online causal softmax: two sets of one warp per TMEM lane quadrant,
+// set a reading accumulator a, so the sets alternate tiles and one set's loads and stores
+// overlap the other's exponentials. Because a row's normaliser is known only after its last
+// tile, each thread writes its
 // per-(row, key block) partial sums with the running maximum they were taken against into the
 // CTA's scratch slot. Four more warps then rescale them once the rows are complete and reduce
 // the m sampled rows of each block row with warp shuffles, while the epilogue warps go on to the
@@ -147,7 +149,7 @@ __global__ void __launch_bounds__(512, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&acc_full[a], 1);
-      mbar_init(&acc_empty[a], 256);
+      mbar_init(&acc_empty[a], 128);   // the four epilogue warps of set a
       mbar_init(&fp_full[a], 256);
       mbar_init(&fp_empty[a], 128);
     }
@@ -248,8 +250,10 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, qph = 0, aph = 0;
-      int acc = 0;
+      uint32_t phase = 0, qph = 0;
+      // key tile n of an item goes to accumulator n & 1 (so the epilogue set that reads a tile
+      // depends on the tile alone, not on the CTA's earlier items); one phase per accumulator
+      uint32_t aph[2] = {0, 0};
       bool ok = true;
       const uint32_t q_base = smem_u32(sQ);
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -257,7 +261,8 @@ __global__ void __launch_bounds__(512, 1)
         est_decode(p, item, bh, t);
         if constexpr (XA) {
           for (int n = 0; n <= t && ok; ++n) {
-            if (!mbar_wait(&acc_empty[acc], aph ^ 1, s_abort, p.status)) {
+            const int acc = n & 1;
+            if (!mbar_wait(&acc_empty[acc], aph[acc] ^ 1, s_abort, p.status)) {
               ok = false;
               break;
             }
@@ -286,17 +291,15 @@ __global__ void __launch_bounds__(512, 1)
             }
             if (!ok) break;
             mma_commit(&acc_full[acc]);
-            if (++acc == 2) {
-              acc = 0;
-              aph ^= 1;
-            }
+            aph[acc] ^= 1;
           }
           continue;
         }
         if (!mbar_wait(q_full, qph, s_abort, p.status)) break;
         qph ^= 1;
         for (int n = 0; n <= t; ++n) {
-          if (!mbar_wait(&acc_empty[acc], aph ^ 1, s_abort, p.status) ||
+          const int acc = n & 1;
+          if (!mbar_wait(&acc_empty[acc], aph[acc] ^ 1, s_abort, p.status) ||
               !mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
             ok = false;
             break;
@@ -321,10 +324,7 @@ __global__ void __launch_bounds__(512, 1)
             stage = 0;
             phase ^= 1;
           }
-          if (++acc == 2) {
-            acc = 0;
-            aph ^= 1;
-          }
+          aph[acc] ^= 1;
         }
         if (ok) mma_commit(q_empty);
       }
@@ -333,12 +333,16 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ softmax / mass epilogue
+    // Two sets of four warps, one warp per TMEM lane quadrant in each. Set a takes the key tiles
+    // n with n & 1 == a, which the MMA warp puts in accumulator a, all 128 columns as two
+    // 64-column halves, so one set's TMEM loads and stores overlap the other set's
+    // exponentials. The split depends on n alone, so a row's result does not depend on which
+    // CTA ran its item.
     const int quad = warp & 3;            // TMEM lanes 32*quad .. 32*quad+31
-    const int half = (warp - 4) >> 2;     // accumulator columns 64*half .. 64*half+63
+    const int set = (warp - 4) >> 2;      // accumulator read by this set
     const int r = quad * 32 + lane;       // row of the 128-row query tile
     const float NEG_INF = -INFINITY;
-    int acc = 0;
-    uint32_t aph = 0;
+    uint32_t aph = 0;                     // phase of accumulator `set`
     bool dead = false;
     int kit = 0;   // this CTA's item ordinal; its scratch buffer is kit & 1
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++kit) {
@@ -359,72 +363,75 @@ __global__ void __launch_bounds__(512, 1)
       const bool row_ok = i < p.ns;
       float m_run = NEG_INF, l_run = 0.f;
       for (int n = 0; n <= t; ++n) {
-        if (!dead) dead = !mbar_wait_warp(&acc_full[acc], aph, s_abort, p.status);
-        float e[SEG];
+        if ((n & 1) != set) continue;   // the other set's tile
+        if (!dead) dead = !mbar_wait_warp(&acc_full[set], aph, s_abort, p.status);
+        aph ^= 1;
+        const uint32_t taddr0 = tmem + (static_cast<uint32_t>(quad * 32) << 16) + set * 128;
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
+          float e[SEG];
 #pragma unroll
-        for (int s = 0; s < SEG; ++s) e[s] = 0.f;
-        if (!dead) {
-          tc_fence_after();
-          uint32_t u[64];
-          const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + acc * 128 +
-                                 half * 64;
-          tmem_ld32(taddr, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-          tmem_ld32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-          tmem_ld_wait();
-          tc_fence_before();
-          mbar_arrive(&acc_empty[acc]);
-          if (row_ok) {
-            float *uf = reinterpret_cast<float *>(u);
-            if (n == t) {   // diagonal key tile: stride j is visible to sampled query i iff j <= i
-              const int j0 = n * 128 + half * 64;
-#pragma unroll
-              for (int c = 0; c < 64; ++c)
-                if (j0 + c > i) uf[c] = -INFINITY;
+          for (int s = 0; s < SEG; ++s) e[s] = 0.f;
+          if (!dead) {
+            tc_fence_after();
+            uint32_t u[64];
+            tmem_ld32(taddr0 + half * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+            tmem_ld32(taddr0 + half * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+            tmem_ld_wait();
+            if (half == 1) {   // both halves read: the MMA may overwrite the accumulator
+              tc_fence_before();
+              mbar_arrive(&acc_empty[set]);
             }
-            float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+            if (row_ok) {
+              float *uf = reinterpret_cast<float *>(u);
+              if (n == t) {   // diagonal key tile: stride j is visible to query i iff j <= i
+                const int j0 = n * 128 + half * 64;
 #pragma unroll
-            for (int c = 0; c < 64; c += 8) {
-              mx[0] = fmax3(mx[0], uf[c], uf[c + 1]);
-              mx[1] = fmax3(mx[1], uf[c + 2], uf[c + 3]);
-              mx[2] = fmax3(mx[2], uf[c + 4], uf[c + 5]);
-              mx[3] = fmax3(mx[3], uf[c + 6], uf[c + 7]);
-            }
-            const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * p.scale_log2;
-            if (tmax > m_run) {
-              l_run *= fast_exp2(m_run - tmax);    // m_run = -inf: exp2(-inf) = 0
-              m_run = tmax;
-            }
-            if (m_run > NEG_INF) {
-              const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
-              const uint64_t negm = f2_pack(-m_run, -m_run);
-              uint64_t tot = 0;
-#pragma unroll
-              for (int s = 0; s < SEG; ++s) {
-                uint64_t acc2 = 0;
-#pragma unroll
-                for (int c = 0; c < M; c += 2) {
-                  const uint64_t xy = ffma2(f2_pack(uf[s * M + c], uf[s * M + c + 1]), sl2, negm);
-                  acc2 = fadd2(acc2, f2_pack(fast_exp2(f2_lo(xy)), fast_exp2(f2_hi(xy))));
-                }
-                e[s] = f2_lo(acc2) + f2_hi(acc2);
-                tot = fadd2(tot, acc2);
+                for (int c = 0; c < 64; ++c)
+                  if (j0 + c > i) uf[c] = -INFINITY;
               }
-              l_run += f2_lo(tot) + f2_hi(tot);
+              float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+#pragma unroll
+              for (int c = 0; c < 64; c += 8) {
+                mx[0] = fmax3(mx[0], uf[c], uf[c + 1]);
+                mx[1] = fmax3(mx[1], uf[c + 2], uf[c + 3]);
+                mx[2] = fmax3(mx[2], uf[c + 4], uf[c + 5]);
+                mx[3] = fmax3(mx[3], uf[c + 6], uf[c + 7]);
+              }
+              const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * p.scale_log2;
+              if (tmax > m_run) {
+                l_run *= fast_exp2(m_run - tmax);    // m_run = -inf: exp2(-inf) = 0
+                m_run = tmax;
+              }
+              if (m_run > NEG_INF) {
+                const uint64_t sl2 = f2_pack(p.scale_log2, p.scale_log2);
+                const uint64_t negm = f2_pack(-m_run, -m_run);
+                uint64_t tot = 0;
+#pragma unroll
+                for (int s = 0; s < SEG; ++s) {
+                  uint64_t acc2 = 0;
+#pragma unroll
+                  for (int c = 0; c < M; c += 2) {
+                    const uint64_t xy =
+                        ffma2(f2_pack(uf[s * M + c], uf[s * M + c + 1]), sl2, negm);
+                    acc2 = fadd2(acc2, f2_pack(fast_exp2(f2_lo(xy)), fast_exp2(f2_hi(xy))));
+                  }
+                  e[s] = f2_lo(acc2) + f2_hi(acc2);
+                  tot = fadd2(tot, acc2);
+                }
+                l_run += f2_lo(tot) + f2_hi(tot);
+              }
             }
           }
-        }
-        if (++acc == 2) {
-          acc = 0;
-          aph ^= 1;
-        }
-        float *dst = e_base + (static_cast<size_t>(n) * SEG_ROW + half * SEG) * 128;
+          float *dst = e_base + (static_cast<size_t>(n) * SEG_ROW + half * SEG) * 128;
 #pragma unroll
-        for (int s = 0; s < SEG; ++s) dst[s * 128] = e[s];
-        ref_base[(n * 2 + half) * 128] = m_run;
+          for (int s = 0; s < SEG; ++s) dst[s * 128] = e[s];
+          ref_base[(n * 2 + half) * 128] = m_run;
+        }
       }
-      // ---- combine the two half-rows' running max / sum
-      sM[half * 128 + r] = m_run;
-      sL[half * 128 + r] = l_run;
+      // ---- combine the two sets' running max / sum of the row
+      sM[set * 128 + r] = m_run;
+      sL[set * 128 + r] = l_run;
       named_bar_sync(1, 256);
       const float m0 = sM[r], m1 = sM[128 + r];
       const float mx = fmaxf(m0, m1);
@@ -433,11 +440,11 @@ __global__ void __launch_bounds__(512, 1)
       if (m1 > NEG_INF) ltot += sL[128 + r] * fast_exp2(m1 - mx);
       named_bar_sync(1, 256);
       const float inv = (row_ok && ltot > 0.f) ? 1.f / ltot : 0.f;
-      if (half == 0) {
+      if (set == 0) {
         sRow[buf * 256 + r] = mx;
         sRow[buf * 256 + 128 + r] = inv;
       }
-      // publishes this thread's partial sums and, for half 0, the row's max and 1 / sum
+      // publishes this thread's partial sums and, for set 0, the row's max and 1 / sum
       mbar_arrive(&fp_full[buf]);
     }
     tc_fence_before();
