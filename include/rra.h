@@ -24,9 +24,11 @@
  *     `kept_cnt` int32 [batch, heads_q, NB] is the length of each kept row.
  *   - Each estimated block row sums to 1: mass(I, J) = (1/m) sum over the m = block/stride
  *     sampled queries i of row I of the stride-softmax probabilities of the strides in block J.
- *   - All pointers are DEVICE pointers, 16-byte aligned, owned by the caller. The library never
- *     allocates or frees memory; all work is enqueued on `stream` (a cudaStream_t; NULL = legacy
- *     default stream) and returns without synchronising, except rra_check_device_status.
+ *   - All pointers are DEVICE pointers, 16-byte aligned, owned by the caller, except the host
+ *     buffers of rra_prefill_host. The library never allocates or frees memory (rra_prefill_host
+ *     creates two streams and a few events once per device); all work is enqueued on `stream` (a
+ *     cudaStream_t; NULL = legacy default stream) and returns without synchronising, except
+ *     rra_check_device_status.
  *   - Argument errors are reported before anything is enqueued. A failed launch returns
  *     RRA_ERR_CUDA. Kernels never trap: a device-side wait that exceeds its time limit, or an
  *     invalid kept list met by the attention kernel, sets a sticky error word in the workspace,
