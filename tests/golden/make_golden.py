@@ -1,7 +1,7 @@
 """Write tests/golden/tiny_oracle.json from the fp64 oracle alone.
 
-The fixture freezes the oracle's masses, kept lists and a few attention outputs on the seeded
-tiny workload (8 heads, d 64, L 1024, B 128, S 8, shift 0, tau 0.9, scale 1), so that a later
+The fixture freezes the oracle's masses, kept lists, a few attention outputs and the XAttention
+estimator's masses on the seeded tiny workload (8 heads, d 64, L 1024, B 128, S 8, shift 0, tau 0.9, scale 1), so that a later
 change to the oracle's arithmetic shows up as a diff of this file. Inputs come from the seeded
 generator; every stored value comes from ``oracle``.
 
@@ -30,6 +30,7 @@ def main():
     mass = orc.estimate(q, k, w.block, w.stride, w.shift, w.softmax_scale)
     idx, cnt = orc.select(mass, nb, w.tau)
     o = orc.sparse_attention(q, k, v, idx, cnt, w.block, w.softmax_scale, rows=SAMPLE_ROWS)
+    xa = orc.xattn_estimate(q, k, w.block, w.stride, w.softmax_scale)
     out = {
         "source": "oracle (fp64) on the seeded tiny workload; written by make_golden.py",
         "workload": w.name, "block": w.block, "stride": w.stride, "shift": w.shift,
@@ -37,6 +38,7 @@ def main():
         "mass": [[float(x) for x in mass[0, h]] for h in range(w.heads_q)],
         "kept_cnt": cnt[0].tolist(),
         "kept_idx": idx[0].tolist(),
+        "xattn_mass": [[float(x) for x in xa[0, h]] for h in range(w.heads_q)],
         "attn_samples": [
             {"b": b, "h": h, "I": I, "t": t, "o_first8": [float(x) for x in o[b, h, I * w.block + t, :8]]}
             for (b, h, I) in SAMPLE_ROWS for t in SAMPLE_T],

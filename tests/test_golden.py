@@ -26,3 +26,5 @@ def test_oracle_matches_frozen_tiny_fixture():
     for s in g["attn_samples"]:
         got = o[s["b"], s["h"], s["I"] * g["block"] + s["t"], :8]
         assert np.abs(got - np.array(s["o_first8"])).max() < 1e-12
+    xa = orc.xattn_estimate(q, k, g["block"], g["stride"], g["softmax_scale"])
+    assert np.abs(xa[0] - np.array(g["xattn_mass"])).max() < 1e-12
