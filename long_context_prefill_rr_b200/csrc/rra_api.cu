@@ -1,5 +1,6 @@
 // C ABI of the RRAttention prefill hot path (declared in include/rra.h): argument validation,
-// workspace carve-up and kernel launches. No memory is allocated here.
+// workspace carve-up, kernel launches and the chunked host-buffer pipeline. No memory is
+// allocated here; the host pipeline creates its two streams and events once per device.
 #include <math.h>
 
 #include <algorithm>
