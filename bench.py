@@ -202,6 +202,15 @@ def max_over_ranks(values, device=None):
     return [float(x) for x in t.cpu()]
 
 
+def spread(values) -> dict:
+    """Median and 10th / 90th percentiles (linear interpolation) of per-step timings."""
+    v = np.asarray(list(values), dtype=np.float64)
+    if v.size == 0:
+        return {"p10": None, "p50": None, "p90": None}
+    p10, p50, p90 = np.percentile(v, [10, 50, 90])
+    return {"p10": float(p10), "p50": float(p50), "p90": float(p90)}
+
+
 def sum_over_ranks(values, device=None):
     """Element-wise sum over the process group (identity when there is none)."""
     import torch
@@ -375,6 +384,10 @@ def run_gpu(args, w):
             "data": "synthetic (seeded, shaped like the pages' Llama-3.1-8B 128K workload)",
             "config": _workload_desc(w, f"heads{ws_n}" if sharded else "replicas"),
             "phases_ms": {"estimate": est_avg, "select": sel_avg, "sparse_attn": att_avg},
+            "phases_ms_spread": {"estimate": spread(est_ms), "select": spread(sel_ms),
+                                 "sparse_attn": spread(att_ms),
+                                 "step": spread([a + b + c for a, b, c in
+                                                 zip(est_ms, sel_ms, att_ms)])},
             "density": density,
             "attn_tflops": achieved, "attn_tflops_executed": executed / (att_avg * 1e-3) / 1e12,
             "estimate_gbs": est_bytes / (est_avg * 1e-3) / 1e9,

@@ -28,3 +28,11 @@ def test_reference_arm_prints_one_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert "workload" in d["config"] and d["config"]["workload"].startswith("tiny")
+
+
+def test_spread_reports_median_and_deciles():
+    sys.path.insert(0, ROOT)
+    import bench
+    d = bench.spread([5.0, 1.0, 3.0, 2.0, 4.0])
+    assert d == {"p10": 1.4, "p50": 3.0, "p90": 4.6}
+    assert bench.spread([]) == {"p10": None, "p50": None, "p90": None}
