@@ -14,7 +14,6 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
 
-import numpy as np  # noqa: E402
 
 import oracle as orc  # noqa: E402
 from long_context_prefill_rr_b200 import workloads as wl  # noqa: E402
