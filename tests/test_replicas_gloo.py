@@ -1,5 +1,5 @@
-"""The N > 1 host path of bench.py: independent replicas whose step times are reduced with a
-max over ranks (gloo, world size 2, CPU)."""
+"""The N > 1 host path of bench.py: step times reduced with a max over ranks, whole-job counts
+with a sum over ranks (gloo, world size 2, CPU)."""
 import os
 import socket
 import sys
@@ -27,9 +27,10 @@ def _worker(rank, world, port, out):
     ws, r, local = bench._dist_env()
     assert (ws, r, local) == (world, rank, rank)
     got = bench.max_over_ranks([10.0 + rank, 3.0 - rank])
+    total = bench.sum_over_ranks([1.0 + rank, 100.0])
     dist.barrier()
     dist.destroy_process_group()
-    out.put((rank, got))
+    out.put((rank, (got, total)))
 
 
 def test_max_over_ranks_two_gloo_ranks():
@@ -43,10 +44,11 @@ def test_max_over_ranks_two_gloo_ranks():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    assert res[0] == res[1] == [11.0, 3.0]
+    assert res[0] == res[1] == ([11.0, 3.0], [3.0, 200.0])
 
 
 def test_max_over_ranks_single_process_is_identity():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
+    assert bench.sum_over_ranks([1.5, 2.5]) == [1.5, 2.5]
