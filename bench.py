@@ -76,6 +76,13 @@ def attention_flops(kept_idx: np.ndarray, kept_cnt: np.ndarray, block: int, d: i
     return useful, executed, n_kept
 
 
+def head_density(kept_cnt: np.ndarray) -> dict:
+    """Kept-block density per (batch row, head) of kept_cnt [b, H, NB]: min, median, max."""
+    b, h, nb = kept_cnt.shape
+    per = kept_cnt.sum(axis=2, dtype=np.int64) / (nb * (nb + 1) / 2)
+    return {"min": float(per.min()), "median": float(np.median(per)), "max": float(per.max())}
+
+
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 20 ms while active."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -339,8 +346,8 @@ def run_gpu(args, w):
     e2e_ms = e_start.elapsed_time(e_stop) / e_steps
 
     total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
-    useful, executed, n_kept = attention_flops(idx.cpu().numpy(), cnt.cpu().numpy(), w.block,
-                                               w.head_dim)
+    cnt_host = cnt.cpu().numpy()
+    useful, executed, n_kept = attention_flops(idx.cpu().numpy(), cnt_host, w.block, w.head_dim)
     h2d_bytes = int(hq.numel() + hk.numel() + hv.numel()) * 2
     d2h_bytes = int(hout.numel()) * 2
     # whole-job figures: kept blocks over every rank's heads, bytes every rank moved
@@ -389,6 +396,7 @@ def run_gpu(args, w):
                                  "step": spread([a + b + c for a, b, c in
                                                  zip(est_ms, sel_ms, att_ms)])},
             "density": density,
+            "density_per_head": head_density(cnt_host),
             "attn_tflops": achieved, "attn_tflops_executed": executed / (att_avg * 1e-3) / 1e12,
             "estimate_gbs": est_bytes / (est_avg * 1e-3) / 1e9,
             "estimate_frac_hbm": est_bytes / (est_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],

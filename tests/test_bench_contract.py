@@ -36,3 +36,20 @@ def test_spread_reports_median_and_deciles():
     d = bench.spread([5.0, 1.0, 3.0, 2.0, 4.0])
     assert d == {"p10": 1.4, "p50": 3.0, "p90": 4.6}
     assert bench.spread([]) == {"p10": None, "p50": None, "p90": None}
+
+
+def test_head_density_and_attention_flops():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from long_context_prefill_rr_b200 import workloads as wl
+    idx, cnt = wl.random_kept_lists(1, 2, 4, 0.0, seed=0)       # diagonal only
+    d = bench.head_density(cnt)
+    assert d == {"min": 0.4, "median": 0.4, "max": 0.4}          # 4 of 10 causal blocks
+    useful, executed, n = bench.attention_flops(idx, cnt, 128, 64)
+    assert n == 8 and executed == 4.0 * 64 * 128 * 128 * 8
+    assert useful == 4.0 * 64 * (128 * 129 / 2) * 8              # every kept block is diagonal
+    idx, cnt = wl.random_kept_lists(1, 1, 4, 1.0, seed=0)       # dense causal
+    assert bench.head_density(cnt)["max"] == 1.0
+    useful, _, n = bench.attention_flops(idx, cnt, 128, 64)
+    assert n == 10 and useful == 4.0 * 64 * (128 * 128 * 6 + 128 * 129 / 2 * 4)
