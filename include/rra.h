@@ -147,17 +147,33 @@ rra_status rra_prefill_host(const rra_params *p, const void *q_host, const void 
  * allocations, or that must avoid cudaMalloc / cudaFree because those calls can synchronise the
  * device. Problems whose rra_workspace_bytes exceeds 48 MiB return RRA_ERR_WORKSPACE before
  * anything is enqueued (on a 148-SM B200: a 32-query-head, 8-KV-head, d = 128 layer at S = 8 fits
- * up to 23K tokens). All
- * calls share the one array: calls whose kernels may overlap on the GPU (other streams, other
- * threads) race, so serialise them. The first call on each device looks up the array's device
- * address; make it before any stream capture begins. Allocates nothing. */
+ * up to 23K tokens). All calls share the one array: calls whose kernels may overlap on the GPU
+ * (other streams, other threads) race, so serialise them. The first call on each device looks
+ * up the array's device address and clears its status word; make it before any stream capture
+ * begins. Device-side errors (an expired barrier wait) go to the array's sticky status word,
+ * which rra_static_scratch_status reads and clears. Allocates nothing. */
 rra_status rra_estimate_static_scratch(const rra_params *p, const void *q, const void *k,
                                        float *mass, rra_stream_t stream);
+
+/* Device status of the fixed scratch array used by rra_estimate_static_scratch, which has no
+ * workspace a caller could hand to rra_check_device_status. No counterpart in the paper either.
+ * Synchronises `stream`, reads the array's sticky error word and clears it; returns as
+ * rra_check_device_status does (RRA_ERR_DEVICE_TIMEOUT if a barrier wait of an earlier
+ * static-scratch call expired: that call's masses are then undefined, and calls made since
+ * returned without computing). raw_word may be NULL. Allocates nothing. */
+rra_status rra_static_scratch_status(rra_stream_t stream, uint32_t *raw_word);
 
 /* Synchronises `stream`, reads the workspace error word and clears it. Returns RRA_OK,
  * RRA_ERR_DEVICE_TIMEOUT (a barrier wait expired), RRA_ERR_INVALID_ARG (a kept list was
  * invalid) or RRA_ERR_CUDA. If raw_word is non-NULL the raw word is stored there. */
 rra_status rra_check_device_status(void *workspace, rra_stream_t stream, uint32_t *raw_word);
+
+/* Time limit of the kernels' device-side barrier waits, in nanoseconds, for every call made
+ * after it in this process (default 4 s; 0 restores the default). A diagnostic and test hook:
+ * a very short limit makes a kernel give up waiting, drain the copies and MMAs it has in flight,
+ * set RRA_ERR_DEVICE_TIMEOUT in the status word and return, which is how the timeout path is
+ * exercised without a real hang. */
+void rra_set_wait_limit_ns(uint64_t ns);
 
 /* Static description of a status code. */
 const char *rra_status_string(rra_status s);

@@ -17,7 +17,10 @@ namespace rra {
 constexpr uint32_t kErrTimeout = 1u;   // a bounded barrier wait expired
 constexpr uint32_t kErrBadList = 2u;   // a kept list entry was out of range / not ascending
 
-// A wait that has not completed after this long gives up (sets kErrTimeout and aborts the CTA).
+// Default time limit of a barrier wait: a wait that has not completed after this long gives up
+// (sets kErrTimeout and aborts the CTA). The launchers pass the limit in each kernel's
+// parameters (rra_set_wait_limit_ns can shorten it, for tests of the timeout path); the drain
+// waits that follow an abort always use this default.
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -65,24 +68,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity. Returns false if the CTA is aborting
-// (another role timed out) or if this wait itself exceeded kWaitLimitNs; in the latter case the
+// (another role timed out) or if this wait itself exceeded `limit_ns`; in the latter case the
 // timeout bit is OR-ed into the device status word and the CTA abort flag is raised.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag,
-                                          uint32_t *status) {
+                                          uint32_t *status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   uint32_t n = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((++n & 63u) == 0) {
+    // the clock on every failed poll (a register read), the flags every 16th
+    if (global_timer_ns() - t0 > limit_ns) {
+      atomicOr(status, kErrTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+    if ((++n & 15u) == 0) {
       if (*abort_flag) return false;
       if (*reinterpret_cast<volatile uint32_t *>(status) & kErrTimeout) {
         *abort_flag = 1;   // another CTA already gave up: do not wait out our own limit
-        return false;
-      }
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
-        atomicOr(status, kErrTimeout);
-        *abort_flag = 1;
         return false;
       }
     }
@@ -90,16 +94,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // True if an earlier wait anywhere in the grid (or an earlier call sharing the workspace whose
-// status was not yet read) timed out; kernels then exit at once.
-__device__ __forceinline__ bool grid_timed_out(const uint32_t *status) {
-  return (*reinterpret_cast<const volatile uint32_t *>(status) & kErrTimeout) != 0;
+// status was not yet read) timed out; kernels then exit at once. Thread 0 reads the word and
+// the CTA takes its answer from shared memory, so every thread of the CTA takes the same branch
+// (the word may change while the CTA starts). Contains a __syncthreads.
+__device__ __forceinline__ bool cta_grid_timed_out(const uint32_t *status, volatile int *s_flag) {
+  if (threadIdx.x == 0)
+    *s_flag = (*reinterpret_cast<const volatile uint32_t *>(status) & kErrTimeout) != 0;
+  __syncthreads();
+  return *s_flag != 0;
 }
 
 // Warp-uniform version for warps that go on to issue .sync.aligned tcgen05 instructions: the
 // result is true only if the wait succeeded on every lane.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity,
-                                               volatile int *abort_flag, uint32_t *status) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                               volatile int *abort_flag, uint32_t *status,
+                                               uint64_t limit_ns) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -87,6 +87,7 @@ struct EstParams {
   float *est_e;
   float *est_ref;
   uint32_t *status;
+  uint64_t wait_ns;  // time limit of a barrier wait
 };
 
 // Work items in longest-first order: the first b*hq items are the last query tile of every
@@ -134,11 +135,12 @@ __global__ void __launch_bounds__(512, 1)
   float *sRow = sL + 256;     // [2 buffers][2][128]: row max and 1 / row sum of buffer b's item
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sRow + 512);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+  volatile int *s_flag = reinterpret_cast<volatile int *>(s_tmem + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  if (grid_timed_out(p.status)) return;   // uniform across the CTA
+  if (cta_grid_timed_out(p.status, s_flag)) return;   // the same answer for every thread
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(512, 1)
           // per key tile: S stages of (queries at offset tt, keys at offset S-1-tt)
           for (int n = 0; n <= t && ok; ++n)
             for (int tt = 0; tt < p.S; ++tt) {
-              if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) {
+              if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status, p.wait_ns)) {
                 ok = false;
                 break;
               }
@@ -214,7 +216,7 @@ __global__ void __launch_bounds__(512, 1)
           continue;
         }
         if (issued_q > 0) {
-          if (!mbar_wait(q_empty, qph, s_abort, p.status)) break;
+          if (!mbar_wait(q_empty, qph, s_abort, p.status, p.wait_ns)) break;
           qph ^= 1;
         }
         mbar_arrive_expect_tx(q_full, TILE_BYTES);
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(512, 1)
           tma_load_3d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, o, bh * p.ns + t * 128);
         ++issued_q;
         for (int n = 0; n <= t; ++n) {
-          if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) {
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -240,11 +242,12 @@ __global__ void __launch_bounds__(512, 1)
           }
         }
       }
-      if (*s_abort) {   // let every copy already issued land before the CTA exits
-        if (issued_q > 0) mbar_wait_drain(q_full, (issued_q - 1) & 1);
-        for (int s = 0; s < NSTAGE; ++s)
-          if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
-      }
+      // Let every copy already issued land before the CTA exits. Without an abort each of
+      // these phases has completed already (the MMA warp consumed it); after one, a copy may
+      // still be in flight even though this loop ended normally.
+      if (issued_q > 0) mbar_wait_drain(q_full, (issued_q - 1) & 1);
+      for (int s = 0; s < NSTAGE; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -262,13 +265,13 @@ __global__ void __launch_bounds__(512, 1)
         if constexpr (XA) {
           for (int n = 0; n <= t && ok; ++n) {
             const int acc = n & 1;
-            if (!mbar_wait(&acc_empty[acc], aph[acc] ^ 1, s_abort, p.status)) {
+            if (!mbar_wait(&acc_empty[acc], aph[acc] ^ 1, s_abort, p.status, p.wait_ns)) {
               ok = false;
               break;
             }
             const uint32_t d_tmem = tmem + acc * 128;
             for (int tt = 0; tt < p.S; ++tt) {
-              if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+              if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
                 ok = false;
                 break;
               }
@@ -295,12 +298,12 @@ __global__ void __launch_bounds__(512, 1)
           }
           continue;
         }
-        if (!mbar_wait(q_full, qph, s_abort, p.status)) break;
+        if (!mbar_wait(q_full, qph, s_abort, p.status, p.wait_ns)) break;
         qph ^= 1;
         for (int n = 0; n <= t; ++n) {
           const int acc = n & 1;
-          if (!mbar_wait(&acc_empty[acc], aph[acc] ^ 1, s_abort, p.status) ||
-              !mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+          if (!mbar_wait(&acc_empty[acc], aph[acc] ^ 1, s_abort, p.status, p.wait_ns) ||
+              !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(512, 1)
           p.est_ref + (static_cast<size_t>(blockIdx.x) * 2 + buf) * p.ntiles * 2 * 128 + r;
       // the buffer's previous item (kit - 2) must have been reduced
       if (!dead && kit >= 2)
-        dead = !mbar_wait_warp(&fp_empty[buf], ((kit >> 1) - 1) & 1, s_abort, p.status);
+        dead = !mbar_wait_warp(&fp_empty[buf], ((kit >> 1) - 1) & 1, s_abort, p.status, p.wait_ns);
       int bh, t;
       est_decode(p, item, bh, t);
       const int i = t * 128 + r;          // sampled query (stride) index of this row
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(512, 1)
       float m_run = NEG_INF, l_run = 0.f;
       for (int n = 0; n <= t; ++n) {
         if ((n & 1) != set) continue;   // the other set's tile
-        if (!dead) dead = !mbar_wait_warp(&acc_full[set], aph, s_abort, p.status);
+        if (!dead) dead = !mbar_wait_warp(&acc_full[set], aph, s_abort, p.status, p.wait_ns);
         aph ^= 1;
         const uint32_t taddr0 = tmem + (static_cast<uint32_t>(quad * 32) << 16) + set * 128;
 #pragma unroll 1
@@ -457,7 +460,7 @@ __global__ void __launch_bounds__(512, 1)
     int kit = 0;
     for (int item = blockIdx.x; item < p.n_items; item += gridDim.x, ++kit) {
       const int buf = kit & 1;
-      if (!mbar_wait_warp(&fp_full[buf], (kit >> 1) & 1, s_abort, p.status)) break;
+      if (!mbar_wait_warp(&fp_full[buf], (kit >> 1) & 1, s_abort, p.status, p.wait_ns)) break;
       const float *e_base = p.est_e + (static_cast<size_t>(blockIdx.x) * 2 + buf) * p.ntiles *
                                           SEG_ROW * 128 + r;
       const float *ref_base =
@@ -622,6 +625,7 @@ static EstParams est_params(const Geometry &g, float *mass, float *est_e, float 
   ep.est_e = est_e;
   ep.est_ref = est_ref;
   ep.status = status;
+  ep.wait_ns = wait_limit_ns();
   return ep;
 }
 

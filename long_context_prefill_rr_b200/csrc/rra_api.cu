@@ -4,6 +4,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "rra.h"
@@ -38,6 +39,10 @@ WorkspaceLayout workspace_layout(const Geometry &g, int num_sms) {
   w.total = align_up(off, 256);
   return w;
 }
+
+static std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
+
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 EncodeTiledFn encode_tiled_fn() {
   static EncodeTiledFn fn = nullptr;
@@ -381,6 +386,10 @@ rra_status rra_check_device_status(void *workspace, rra_stream_t stream, uint32_
   if (word & rra::kErrTimeout) return RRA_ERR_DEVICE_TIMEOUT;
   if (word & rra::kErrBadList) return RRA_ERR_INVALID_ARG;
   return RRA_OK;
+}
+
+void rra_set_wait_limit_ns(uint64_t ns) {
+  rra::g_wait_limit_ns.store(ns == 0 ? rra::kWaitLimitNs : ns, std::memory_order_relaxed);
 }
 
 const char *rra_status_string(rra_status s) {

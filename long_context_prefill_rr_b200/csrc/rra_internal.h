@@ -33,6 +33,10 @@ struct WorkspaceLayout {
 
 WorkspaceLayout workspace_layout(const Geometry &g, int num_sms);
 
+// Time limit of the kernels' barrier waits, in ns (kWaitLimitNs unless rra_set_wait_limit_ns
+// set another).
+uint64_t wait_limit_ns();
+
 // Driver entry point for tensor-map encoding (resolved once through the runtime).
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,

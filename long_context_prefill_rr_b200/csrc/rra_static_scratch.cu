@@ -15,8 +15,11 @@
 //     streams, or different host threads) race and corrupt each other's results. Serialise
 //     them, e.g. issue them on one stream.
 //   - The first call on each device looks up the array's device address (a host-side query,
-//     done once per device with that device current); make that first call before any stream
-//     capture begins.
+//     done once per device with that device current) and clears the array's status word; make
+//     that first call before any stream capture begins.
+//   - The status word is sticky, as a workspace's is: a kernel whose barrier wait timed out
+//     sets it, later calls then enqueue kernels that exit at once, and
+//     rra_static_scratch_status reads and clears it.
 #include <mutex>
 
 #include "rra.h"
@@ -36,8 +39,10 @@ static __device__ __align__(256) unsigned char g_rra_static_scratch[kStaticScrat
 std::mutex g_mu;
 void *g_addr[kMaxDevices] = {nullptr};
 
-// Device address of the scratch array on the current device (looked up once per device).
-cudaError_t scratch_address(void **out) {
+// Device address of the scratch array on the current device. The first call on a device looks
+// it up and clears the status word at its start (enqueued on `stream`, ahead of any kernel that
+// reads it).
+cudaError_t scratch_address(void **out, cudaStream_t stream) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -46,6 +51,8 @@ cudaError_t scratch_address(void **out) {
   if (g_addr[dev] == nullptr) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_rra_static_scratch);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(p, 0, 256, stream);
     if (e != cudaSuccess) return e;
     g_addr[dev] = p;
   }
@@ -73,10 +80,17 @@ extern "C" rra_status rra_estimate_static_scratch(const rra_params *p, const voi
   }
   if (need > kStaticScratchBytes) return RRA_ERR_WORKSPACE;
   void *scratch = nullptr;
-  if (scratch_address(&scratch) != cudaSuccess) return RRA_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents; only the status word must start at zero
-  // (pooled keys and partial sums are fully rewritten before they are read).
-  if (cudaMemsetAsync(scratch, 0, 256, st) != cudaSuccess) return RRA_ERR_CUDA;
+  if (scratch_address(&scratch, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RRA_ERR_CUDA;
+  // The array keeps the previous call's contents. Pooled keys and partial sums are rewritten
+  // before they are read; the status word was cleared at set-up and stays set after a timeout
+  // until rra_static_scratch_status reads it.
   return rra_estimate(p, q, k, mass, scratch, need, stream);
+}
+
+extern "C" rra_status rra_static_scratch_status(rra_stream_t stream, uint32_t *raw_word) {
+  void *scratch = nullptr;
+  if (scratch_address(&scratch, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return RRA_ERR_CUDA;
+  return rra_check_device_status(scratch, stream, raw_word);
 }

@@ -42,6 +42,7 @@ struct AttnParams {
   const int32_t *kept_cnt;
   __nv_bfloat16 *out;
   uint32_t *status;
+  uint64_t wait_ns;  // time limit of a barrier wait
 };
 
 // Walks one kept row, yielding the valid entries (0 <= J <= I, strictly ascending). The entry
@@ -162,6 +163,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t *drain = o_final + 2;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+  volatile int *s_flag = reinterpret_cast<volatile int *>(s_tmem + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(384, 1)
     kvrow[x] = (b * p.hkv + (valid[x] ? h : h0) / p.g) * p.L;
   }
 
-  if (grid_timed_out(p.status)) return;   // uniform across the CTA
+  if (cta_grid_timed_out(p.status, s_flag)) return;   // the same answer for every thread
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < NSTAGE; ++s) {
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int s = 0; s < NSTAGE; ++s) issued[s] = 0;
       bool ok = true;
       auto load = [&](const CUtensorMap *map, int row) -> bool {
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status)) return false;
+        if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status, p.wait_ns)) return false;
         mbar_arrive_expect_tx(&kv_full[stage], TILE_BYTES);
         uint8_t *dst = sRing + stage * TILE_BYTES;
         for (int c = 0; c < NCHUNK; ++c)
@@ -266,11 +268,11 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!any) break;
       }
-      if (*s_abort) {
-        if (q_any) mbar_wait_drain(q_full, 0);
-        for (int s = 0; s < NSTAGE; ++s)
-          if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
-      }
+      // Let every copy already issued land before the CTA exits (without an abort these
+      // phases have completed already: the MMA warp consumed them).
+      if (q_any) mbar_wait_drain(q_full, 0);
+      for (int s = 0; s < NSTAGE; ++s)
+        if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(384, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      if (n[0] + n[1] > 0) ok = mbar_wait(q_full, 0, s_abort, p.status);
+      if (n[0] + n[1] > 0) ok = mbar_wait(q_full, 0, s_abort, p.status, p.wait_ns);
       // descriptors: base of each operand; per-MMA offsets are added in 16-byte units
       const uint32_t ring_base = smem_u32(sRing);
       const uint64_t q_desc[2] = {sdesc_kmajor_sw128(smem_u32(sQ)),
@@ -296,8 +298,8 @@ __global__ void __launch_bounds__(384, 1)
           if (j >= 1 && j <= n[x]) {
             // O_x += P_x(j-1) V_x(j-1); P sits in the S columns of item x. Keys 0..63 go in
             // as soon as their half of P is written, while the softmax finishes keys 64..127.
-            if (!mbar_wait(&p_half[x], (j - 1) & 1, s_abort, p.status) ||
-                !mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+            if (!mbar_wait(&p_half[x], (j - 1) & 1, s_abort, p.status, p.wait_ns) ||
+                !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -307,7 +309,7 @@ __global__ void __launch_bounds__(384, 1)
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
                           (j > 1 || kk > 0) ? 1u : 0u);
-            if (!mbar_wait(&p_full[x], (j - 1) & 1, s_abort, p.status)) {
+            if (!mbar_wait(&p_full[x], (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           if (j < n[x]) {
             // S_x = Q_x K_x(j)^T into the same TMEM columns
-            if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status)) {
+            if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
               ok = false;
               break;
             }
@@ -367,7 +369,7 @@ __global__ void __launch_bounds__(384, 1)
     cur.init(p, bh[x], I, valid[x]);
     int t = 0;
     for (int J = cur.next(nullptr); J >= 0; J = cur.next(nullptr), ++t) {
-      if (!mbar_wait_warp(&s_full[x], t & 1, s_abort, p.status)) {
+      if (!mbar_wait_warp(&s_full[x], t & 1, s_abort, p.status, p.wait_ns)) {
         dead = true;
         break;
       }
@@ -454,7 +456,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (valid[x]) {
       __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh[x]) * p.L + I * 128 + r) * D;
-      if (!dead && t > 0 && mbar_wait_warp(&o_final[x], 0, s_abort, p.status)) {
+      if (!dead && t > 0 && mbar_wait_warp(&o_final[x], 0, s_abort, p.status, p.wait_ns)) {
         tc_fence_after();
         const uint64_t s01 = fadd2(lsum[0], lsum[1]), s23 = fadd2(lsum[2], lsum[3]);
         const uint64_t s4 = fadd2(s01, s23);
@@ -557,6 +559,7 @@ cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, 
   ap.kept_cnt = kept_cnt;
   ap.out = static_cast<__nv_bfloat16 *>(out);
   ap.status = status;
+  ap.wait_ns = wait_limit_ns();
   const int64_t grid = static_cast<int64_t>(ap.n_pairs) * g.nb;
   if (g.d == 128) return launch_attn_t<128>(mq, mk, mv, ap, grid, stream);
   if (g.d == 64) return launch_attn_t<64>(mq, mk, mv, ap, grid, stream);

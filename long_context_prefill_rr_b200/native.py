@@ -40,6 +40,8 @@ _SIGS = {
                                                _c.c_void_p, _c.c_void_p]),
     "rra_check_device_status": (_c.c_int, [_c.c_void_p, _c.c_void_p,
                                            _c.POINTER(_c.c_uint32)]),
+    "rra_static_scratch_status": (_c.c_int, [_c.c_void_p, _c.POINTER(_c.c_uint32)]),
+    "rra_set_wait_limit_ns": (None, [_c.c_uint64]),
     "rra_status_string": (_c.c_char_p, [_c.c_int]),
     "rra_version": (_c.c_char_p, []),
 }
@@ -221,6 +223,20 @@ def check_device_status(ws, stream=None) -> tuple[int, int]:
     raw = ctypes.c_uint32(0)
     st = load().rra_check_device_status(_ptr(ws), _stream(stream), ctypes.byref(raw))
     return int(st), int(raw.value)
+
+
+def static_scratch_status(stream=None) -> tuple[int, int]:
+    """(status, raw status word) of the fixed scratch array behind estimate_static_scratch;
+    synchronises the stream and clears the word."""
+    raw = ctypes.c_uint32(0)
+    st = load().rra_static_scratch_status(_stream(stream), ctypes.byref(raw))
+    return int(st), int(raw.value)
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Time limit of the kernels' barrier waits for later calls (0 restores the 4 s default);
+    a test hook for the timeout path."""
+    load().rra_set_wait_limit_ns(int(ns))
 
 
 def prefill_host(p: RraParams, q_host, k_host, v_host, out_host, q_dev, k_dev, v_dev, out_dev,

@@ -23,3 +23,18 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Print the GPU parity records (rows checked, mass error, kept-list mismatches excused by
+    the 1e-4 boundary rule, attention error) so they reach the log without -s."""
+    mod = sys.modules.get("parity")
+    recs = getattr(mod, "RECORDS", None) if mod else None
+    if not recs:
+        return
+    tr = terminalreporter
+    tr.section("parity against the fp64 oracle")
+    for r in recs:
+        fields = " ".join(f"{k}={v:.3g}" if isinstance(v, float) else f"{k}={v}"
+                          for k, v in r.items() if k not in ("label", "when"))
+        tr.write_line(f"{r['label']}: {fields}")

@@ -1,0 +1,58 @@
+"""The fp64 oracle over many heads at once, on a pool of spawned processes (test helper).
+
+Spawned, not forked: the test process holds a CUDA context, and a child forked from it hangs.
+This module imports only numpy, the oracle and the input generator, so the workers start
+quickly; each worker uses a single BLAS thread and computes every block row of one head.
+"""
+from __future__ import annotations
+
+import concurrent.futures
+import multiprocessing
+import os
+
+import numpy as np
+
+import oracle as orc
+from long_context_prefill_rr_b200 import workloads as wl
+
+
+def head_masses(args):
+    """fp64 oracle masses of every block row of one (batch, head): [NB(NB+1)/2]."""
+    q_bits, k_bits, h, nb, block, stride, shift, scale = args
+    q = wl.bf16_bits_to_f64(q_bits)
+    kbar = orc.pooled_keys(wl.bf16_bits_to_f64(k_bits), stride)
+    out = np.empty(orc.tri_offset(nb), dtype=np.float64)
+    for I in range(nb):
+        out[orc.tri_offset(I):orc.tri_offset(I + 1)] = orc.estimate_block_row(
+            q, kbar, h, I, block, stride, shift, scale)
+    return out
+
+
+def masses_full(q_bits, k_bits, batch, heads_q, heads_kv, seqlen, block, stride, shift, scale,
+                heads=None, workers=None) -> dict:
+    """{(b, h): masses of every block row} for every (b, h), or the listed ones."""
+    nb = seqlen // block
+    keys = heads if heads is not None else [(b, h) for b in range(batch) for h in range(heads_q)]
+    tasks = [(np.ascontiguousarray(q_bits[b, h]),
+              np.ascontiguousarray(k_bits[b, orc.kv_head(h, heads_q, heads_kv)]),
+              h, nb, block, stride, shift, scale) for b, h in keys]
+    if workers is None:
+        # below 64K tokens a head takes well under a second: starting workers costs more
+        workers = 1 if seqlen < 65536 else max(1, min(len(tasks), len(os.sched_getaffinity(0))))
+    if workers == 1 or len(tasks) == 1:
+        return {key: head_masses(t) for key, t in zip(keys, tasks)}
+    names = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+    saved = {v: os.environ.get(v) for v in names}
+    for v in names:
+        os.environ[v] = "1"
+    try:
+        ctx = multiprocessing.get_context("spawn")
+        with concurrent.futures.ProcessPoolExecutor(workers, mp_context=ctx) as ex:
+            res = list(ex.map(head_masses, tasks))
+    finally:
+        for v, old in saved.items():
+            if old is None:
+                os.environ.pop(v, None)
+            else:
+                os.environ[v] = old
+    return dict(zip(keys, res))

@@ -1,8 +1,10 @@
 """rra_prefill_host: host buffers in and out, chunked so that the copies overlap the compute.
-Its kept lists and output equal rra_prefill's on the same inputs, bit for bit. The chunks are
-independent sub-problems: query-head groups within a KV head, whole KV heads when there are more
-than 16, or batch rows. A chunk of heads runs with the round-robin shift advanced by its first
-head. The cases cover each kind of chunk."""
+The chunks are independent sub-problems: query-head groups within a KV head, whole KV heads when
+there are more than 16, or batch rows. A chunk of heads runs with the round-robin shift advanced
+by its first head (the sampled offset rotates across heads: RRAttention abstract). Its kept lists
+and output are compared with the fp64 oracle run on the global heads and shift (kept lists of
+every row under the boundary rule, output rows sampled), and must equal rra_prefill's on the
+same inputs bit for bit. The cases cover each kind of chunk."""
 import numpy as np
 import pytest
 import torch
@@ -50,6 +52,20 @@ def test_prefill_host_equals_prefill(cuda_device, name):
         torch.cuda.current_stream().synchronize()
         st, raw = native.check_device_status(ws)
         assert st == 0, raw
-        assert np.array_equal(idx.cpu().numpy(), ref["idx"])
-        assert np.array_equal(cnt.cpu().numpy(), ref["cnt"])
-        assert np.array_equal(oh.float().numpy(), ref["out"])
+        got = dict(idx=idx.cpu().numpy(), cnt=cnt.cpu().numpy(), out=oh.float().numpy())
+        assert np.array_equal(got["idx"], ref["idx"])
+        assert np.array_equal(got["cnt"], ref["cnt"])
+        assert np.array_equal(got["out"], ref["out"])
+    # against the oracle on the global heads (the masses stay in the workspace: the lists are
+    # checked against the oracle's select on the oracle's masses)
+    nb = w.seqlen // w.block
+    full = par.oracle_masses_full(qb, kb, p)
+    mism, exc, n = par.compare_select_rows(got, par.mass_rows(full, nb), w.tau)
+    assert not mism, f"{name}: kept-list mismatches outside the boundary rule: {mism[:5]}"
+    qc, kc, vc = par.HeadCache(qb), par.HeadCache(kb), par.HeadCache(vb)
+    rows = par.sample_rows(p, 24, seed=7)
+    ref_rows = par.oracle_attention_rows(qc, kc, vc, p, got["idx"], got["cnt"], rows)
+    ma, rr = par.attention_rows_errors(got["out"], ref_rows)
+    assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (name, ma, rr)
+    par.record(f"prefill_host_{name}", list_rows=n, list_mismatch_excused=len(exc),
+               attn_rows=f"sampled {len(rows)}", attn_max_abs=ma, attn_rel_rms=rr)

@@ -1,7 +1,10 @@
-"""Head-sharded layers on the GPU: each shard of a layer, run through the C ABI with its own
-head counts and shifted round-robin shift, gives exactly (bit for bit) the masses, kept lists
-and attention output the whole-layer run gives for those heads. The shards run one after another
-on one device, as W ranks would each run theirs."""
+"""Head-sharded layers on the GPU. Each shard of a layer runs through the C ABI with its own head
+counts and the round-robin shift advanced by its first query head (the offset rotates across
+heads: RRAttention abstract, "rotating query sampling positions across attention heads within
+each stride"). The shards run one after another on one device, as W ranks would each run
+theirs. Their outputs, put back at their global head positions, are compared with the fp64
+oracle run on the GLOBAL heads and shift (every mass and kept list; every output row for the
+tiny case, sampled rows otherwise), and must equal the whole-layer run bit for bit."""
 import numpy as np
 import pytest
 
@@ -20,16 +23,25 @@ CASES = {
 
 @pytest.mark.parametrize("name,world", [("tiny_gqa", 2), ("tiny_gqa", 4), ("llama8k", 2),
                                         ("llama8k", 8), ("video_short", 4)])
-def test_shards_reproduce_the_whole_layer(cuda_device, name, world):
+def test_shards_match_the_oracle_and_the_whole_layer(cuda_device, name, world):
     w, p = par.workload_params(CASES[name])
     qb, kb, vb = wl.make_workload(w)
     full = par.run_prefill(p, par.to_dev(qb), par.to_dev(kb), par.to_dev(vb))
     assert full["status"] == 0, full["raw"]
+    joined = {key: np.zeros_like(full[key]) for key in ("mass", "idx", "cnt", "out")}
     for r in range(world):
         ps, s = sharding.shard_params(p, r, world)
         part = par.run_prefill(ps, par.to_dev(sharding.take_heads(qb, s.q0, s.q1)),
                                par.to_dev(sharding.take_heads(kb, s.kv0, s.kv1)),
                                par.to_dev(sharding.take_heads(vb, s.kv0, s.kv1)))
         assert part["status"] == 0, part["raw"]
-        for key in ("mass", "idx", "cnt", "out"):
-            assert np.array_equal(part[key], full[key][:, s.q0:s.q1]), (name, world, r, key)
+        for key in joined:
+            joined[key][:, s.q0:s.q1] = part[key]
+    joined["status"], joined["raw"] = 0, 0
+    label = f"shards_{name}_w{world}"
+    if name == "tiny_gqa":
+        par.full_check(w, p, (qb, kb, vb), joined, label)
+    else:
+        par.long_check(w, p, (qb, kb, vb), joined, label, attn_rows=24, seed=world)
+    for key in ("mass", "idx", "cnt", "out"):
+        assert np.array_equal(joined[key], full[key]), (name, world, key)
