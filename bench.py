@@ -453,17 +453,15 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
+        # steps 1 + 2 in one launch (the estimate kernel also selects), then step 3
         if ev is not None:
             ev[0].record(stream)
-        native.estimate(p, q, k, mass, wsp)
+        native.estimate_select(p, q, k, idx, cnt, wsp, mass=mass)
         if ev is not None:
             ev[1].record(stream)
-        native.select(p, mass, idx, cnt)
-        if ev is not None:
-            ev[2].record(stream)
         native.sparse_attn(p, q, k, v, idx, cnt, out, wsp)
         if ev is not None:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -471,7 +469,7 @@ def run_gpu(args, w):
     st, raw = native.check_device_status(wsp)
     if st != 0:
         raise RuntimeError(f"device status {raw:#x} after warm-up")
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws_n > 1:
         dist.barrier()
@@ -485,9 +483,8 @@ def run_gpu(args, w):
     if ws_n > 1:
         dist.barrier()
     total_ms = start.elapsed_time(stop)
-    est_ms = [e[0].elapsed_time(e[1]) for e in events]
-    sel_ms = [e[1].elapsed_time(e[2]) for e in events]
-    att_ms = [e[2].elapsed_time(e[3]) for e in events]
+    es_ms = [e[0].elapsed_time(e[1]) for e in events]
+    att_ms = [e[1].elapsed_time(e[2]) for e in events]
     st, raw = native.check_device_status(wsp)
     if st != 0:
         raise RuntimeError(f"device status {raw:#x} after the timed steps")
@@ -521,8 +518,7 @@ def run_gpu(args, w):
         heads_all = w.heads_q * (1 if sharded else ws_n)
         density = n_kept_all / (w.batch * heads_all * nb * (nb + 1) / 2)
         att_avg = float(np.mean(att_ms))
-        est_avg = float(np.mean(est_ms))
-        sel_avg = float(np.mean(sel_ms))
+        es_avg = float(np.mean(es_ms))
         achieved = useful / (att_avg * 1e-3) / 1e12
         # a timed region under 2 s is a burst: the burst GEMM peak applies; a longer one runs
         # into the power cap, where the sustained peak applies
@@ -561,19 +557,17 @@ def run_gpu(args, w):
             "vs_baseline": None, "dtype": "bf16",
             "data": f"synthetic (seeded, shaped like the pages' workloads: {w.name})",
             "config": _workload_desc(w, f"heads{ws_n}" if sharded else "replicas"),
-            "phases_ms": {"estimate": est_avg, "select": sel_avg, "sparse_attn": att_avg},
-            "phases_ms_spread": {"estimate": spread(est_ms), "select": spread(sel_ms),
-                                 "sparse_attn": spread(att_ms),
-                                 "step": spread([a + b + c for a, b, c in
-                                                 zip(est_ms, sel_ms, att_ms)])},
+            "phases_ms": {"estimate_select": es_avg, "sparse_attn": att_avg},
+            "phases_ms_spread": {"estimate_select": spread(es_ms), "sparse_attn": spread(att_ms),
+                                 "step": spread([a + b for a, b in zip(es_ms, att_ms)])},
+            "phases_note": "estimate and select run in one kernel (rra_estimate_select); "
+                           "the pooled-key kernel is counted with them",
             "density": density,
             "density_per_head": head_density(cnt_host),
             "attn_tflops": achieved, "attn_tflops_executed": executed / (att_avg * 1e-3) / 1e12,
-            "estimate_gbs": est_bytes / (est_avg * 1e-3) / 1e9,
-            "estimate_frac_hbm": est_bytes / (est_avg * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "select_gbs": sel_bytes / (sel_avg * 1e-3) / 1e9,
-            "estimate_select_frac_hbm": (est_bytes + sel_bytes) / ((est_avg + sel_avg) * 1e-3)
-            / 1e9 / peaks["hbm_gbs"],
+            "estimate_select_gbs": (est_bytes + sel_bytes) / (es_avg * 1e-3) / 1e9,
+            "estimate_select_frac_hbm": (est_bytes + sel_bytes) / (es_avg * 1e-3) / 1e9
+            / peaks["hbm_gbs"],
             "roofline": {"bound": "tensor", "kernel": "bs_attn_fwd_kernel", "achieved": achieved,
                          "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{peaks['source']} bf16 "
@@ -585,7 +579,7 @@ def run_gpu(args, w):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_ms if sharded else e2e_ms / ws_n, "unit": UNIT,
                     "h2d_bytes_per_step": int(h2d_all), "d2h_bytes_per_step": int(d2h_all)},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": 3 * args.steps,
             "e2e_api": "rra_prefill_host (pinned host buffers; copies overlapped with the "
                        "compute, chunk by chunk)",
             "clocks": clocks.summary(),

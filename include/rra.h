@@ -82,6 +82,13 @@ size_t rra_workspace_bytes(const rra_params *p);
 rra_status rra_estimate(const rra_params *p, const void *q, const void *k, float *mass,
                         void *workspace, size_t workspace_bytes, rra_stream_t stream);
 
+/* Steps 1 and 2: rra_estimate followed by rra_select on its masses, in one call. mass may be
+ * NULL (then the masses live in the workspace, which rra_workspace_bytes accounts for);
+ * kept_idx / kept_cnt as rra_select writes them. */
+rra_status rra_estimate_select(const rra_params *p, const void *q, const void *k, float *mass,
+                               int32_t *kept_idx, int32_t *kept_cnt, void *workspace,
+                               size_t workspace_bytes, rra_stream_t stream);
+
 /* Step 1, alternative estimator (the XAttention review, sections 2-3: antidiagonal scoring
  * with stride-level softmax): the same mass output and layout as rra_estimate, but the
  * stride-level score of query stride i against key stride j is the sum of the S logits on the

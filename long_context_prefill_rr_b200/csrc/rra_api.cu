@@ -128,14 +128,20 @@ T *ws_at(void *ws, size_t off) {
   return reinterpret_cast<T *>(static_cast<uint8_t *>(ws) + off);
 }
 
+// Pooled keys, then the estimate kernel; with kept_idx / kept_cnt, then the select kernel. (A
+// select fused into the estimate kernel's reduction warps was measured slower at every size:
+// the bisection then runs on 4 warps per SM instead of a grid of its own.)
 rra_status run_estimate(const Geometry &g, const void *q, const void *k, float *mass, void *ws,
-                        const WorkspaceLayout &w, int sms, cudaStream_t st) {
+                        const WorkspaceLayout &w, int sms, cudaStream_t st,
+                        int32_t *kept_idx = nullptr, int32_t *kept_cnt = nullptr) {
   cudaError_t e = rra::launch_pool_keys(g, k, ws_at<void>(ws, w.khi), ws_at<void>(ws, w.klo),
                                         sms, st);
   if (e != cudaSuccess) return RRA_ERR_CUDA;
   e = rra::launch_rr_estimate(g, q, ws_at<void>(ws, w.khi), ws_at<void>(ws, w.klo), mass,
                               ws_at<float>(ws, w.est_e), ws_at<float>(ws, w.est_ref),
                               w.est_slots, status_word(ws, w), st);
+  if (e == cudaSuccess && kept_idx != nullptr)
+    e = rra::launch_topt_select(g, mass, kept_idx, kept_cnt, sms, st);
   return cuda_status(e);
 }
 
@@ -143,10 +149,8 @@ rra_status run_prefill(const Geometry &g, const void *q, const void *k, const vo
                        float *mass, int32_t *kept_idx, int32_t *kept_cnt, void *workspace,
                        const WorkspaceLayout &w, int sms, cudaStream_t st) {
   float *m = mass ? mass : ws_at<float>(workspace, w.mass);
-  rra_status s = run_estimate(g, q, k, m, workspace, w, sms, st);
+  rra_status s = run_estimate(g, q, k, m, workspace, w, sms, st, kept_idx, kept_cnt);
   if (s != RRA_OK) return s;
-  if (rra::launch_topt_select(g, m, kept_idx, kept_cnt, sms, st) != cudaSuccess)
-    return RRA_ERR_CUDA;
   return cuda_status(rra::launch_sparse_attn(g, q, k, v, kept_idx, kept_cnt, out,
                                              status_word(workspace, w), st));
 }
@@ -208,6 +212,25 @@ rra_status rra_estimate(const rra_params *p, const void *q, const void *k, float
   const WorkspaceLayout w = rra::workspace_layout(g, sms);
   if (workspace_bytes < w.total) return RRA_ERR_WORKSPACE;
   return run_estimate(g, q, k, mass, workspace, w, sms, reinterpret_cast<cudaStream_t>(stream));
+}
+
+rra_status rra_estimate_select(const rra_params *p, const void *q, const void *k, float *mass,
+                               int32_t *kept_idx, int32_t *kept_cnt, void *workspace,
+                               size_t workspace_bytes, rra_stream_t stream) {
+  Geometry g;
+  rra_status s = resolve(p, kNeedsStride | kNeedsHeadDim, &g);
+  if (s != RRA_OK) return s;
+  if (empty(g)) return RRA_OK;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(kept_idx) || !ptr_ok(kept_cnt) ||
+      !ptr_ok(workspace) || (mass != nullptr && !ptr_ok(mass)))
+    return RRA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return RRA_ERR_CUDA;
+  const WorkspaceLayout w = rra::workspace_layout(g, sms);
+  if (workspace_bytes < w.total) return RRA_ERR_WORKSPACE;
+  float *m = mass ? mass : ws_at<float>(workspace, w.mass);
+  return run_estimate(g, q, k, m, workspace, w, sms, reinterpret_cast<cudaStream_t>(stream),
+                      kept_idx, kept_cnt);
 }
 
 rra_status rra_estimate_xattn(const rra_params *p, const void *q, const void *k, float *mass,

@@ -34,6 +34,9 @@ _SIGS = {
                                _c.c_void_p]),
     "rra_prefill_host": (_c.c_int, [_c.c_void_p] + [_c.c_void_p] * 11 + [_c.c_size_t,
                                                                           _c.c_void_p]),
+    "rra_estimate_select": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
+                                       _c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_size_t,
+                                       _c.c_void_p]),
     "rra_estimate_xattn": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p, _c.c_void_p,
                                       _c.c_void_p, _c.c_size_t, _c.c_void_p]),
     "rra_estimate_static_scratch": (_c.c_int, [_c.c_void_p, _c.c_void_p, _c.c_void_p,
@@ -152,6 +155,22 @@ def estimate(p: RraParams, q, k, mass, ws, stream=None):
     _expect(mass, torch.float32, sh["mass"], "mass")
     _check(load().rra_estimate(_p(p), _ptr(q), _ptr(k), _ptr(mass), _ptr(ws), ws.numel(),
                                _stream(stream)), "rra_estimate")
+
+
+def estimate_select(p: RraParams, q, k, kept_idx, kept_cnt, ws, mass=None, stream=None):
+    """Steps 1 and 2 in one launch (rra_estimate_select): masses (into ``mass``, or the
+    workspace when None) and the kept lists of rra_select."""
+    import torch
+    sh = shapes(p)
+    _expect(q, torch.bfloat16, sh["q"], "q")
+    _expect(k, torch.bfloat16, sh["kv"], "k")
+    _expect(kept_idx, torch.int32, sh["kept_idx"], "kept_idx")
+    _expect(kept_cnt, torch.int32, sh["kept_cnt"], "kept_cnt")
+    if mass is not None:
+        _expect(mass, torch.float32, sh["mass"], "mass")
+    _check(load().rra_estimate_select(_p(p), _ptr(q), _ptr(k), _ptr(mass), _ptr(kept_idx),
+                                      _ptr(kept_cnt), _ptr(ws), ws.numel(), _stream(stream)),
+           "rra_estimate_select")
 
 
 def estimate_xattn(p: RraParams, q, k, mass, ws, stream=None):

@@ -28,7 +28,7 @@ def lib():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
-        "rra_workspace_bytes", "rra_estimate", "rra_select", "rra_sparse_attn", "rra_prefill",
+        "rra_workspace_bytes", "rra_estimate", "rra_estimate_select", "rra_select", "rra_sparse_attn", "rra_prefill",
         "rra_estimate_static_scratch", "rra_estimate_xattn", "rra_prefill_host",
         "rra_check_device_status", "rra_static_scratch_status", "rra_set_wait_limit_ns",
         "rra_status_string", "rra_version"])

@@ -225,3 +225,33 @@ def test_llama128k_parity(cuda_device):
     del dev
     torch.cuda.empty_cache()
     par.long_check(w, p, bits, gpu, "llama128k", attn_rows=96, seed=3)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", {}),
+    ("tiny", dict(stride=4, tau=0.5, heads_q=8, heads_kv=2, head_dim=128, seqlen=1152)),
+    ("tiny", dict(stride=32, tau=1.0)),
+    ("llama8k", {}),
+    ("llama32k", dict(stride=16, tau=0.95)),
+])
+def test_estimate_select_equals_estimate_then_select(cuda_device, name, over):
+    """rra_estimate_select (steps 1 and 2 in one call) gives the masses and kept lists of
+    rra_estimate followed by rra_select, bit for bit, with the masses in a caller buffer or kept
+    in the workspace."""
+    w, p = par.workload_params(wl.WORKLOADS[name], **over)
+    bits, (q, k, _) = _prepare(w)
+    sh = native.shapes(p)
+    m1 = torch.empty(sh["mass"], dtype=torch.float32, device="cuda")
+    i1 = torch.empty(sh["kept_idx"], dtype=torch.int32, device="cuda")
+    c1 = torch.empty(sh["kept_cnt"], dtype=torch.int32, device="cuda")
+    ws = native.new_workspace(p)
+    native.estimate(p, q, k, m1, ws)
+    native.select(p, m1, i1, c1)
+    m2, i2, c2 = torch.empty_like(m1), torch.full_like(i1, 7), torch.full_like(c1, 7)
+    native.estimate_select(p, q, k, i2, c2, ws, mass=m2)
+    st, raw = native.check_device_status(ws)
+    assert st == 0, raw
+    assert torch.equal(m1, m2) and torch.equal(i1, i2) and torch.equal(c1, c2)
+    i3, c3 = torch.full_like(i1, 7), torch.full_like(c1, 7)
+    native.estimate_select(p, q, k, i3, c3, ws)          # masses kept in the workspace
+    assert torch.equal(i1, i3) and torch.equal(c1, c3)
