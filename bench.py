@@ -725,7 +725,7 @@ def run_search_study(args):
 
 
 # bump when the attention kernel changes, so stale ncu traffic is not reported
-KERNEL_REV = "attn-v3"
+KERNEL_REV = "attn-v5-single"
 
 
 def main(argv=None):

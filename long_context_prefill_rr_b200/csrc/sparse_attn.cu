@@ -2,28 +2,26 @@
 // the selected blocks; "regular block-sparse FlashAttention execution" in the RBS-Attention
 // digest; online softmax as in FlashAttention / FlashAttention-2), GQA head mapping.
 //
-// One CTA runs two work items side by side: query block I of heads 2c and 2c+1 (of one batch
-// row), each with its own kept list. Grid order is longest-first (I descending), by KV-head
-// chunk when K and V exceed L2 (see attn_item). Roles:
-//   warp 0       TMA producer: both Q tiles once, then per step j the tiles V_A(j-1), K_A(j),
-//                V_B(j-1), K_B(j) through a ring of 128-row tiles, in the order the MMA warp
-//                consumes them;
-//   warp 1       MMA issuer (one thread), same order: O_X += P_X V_X(j-1) with P read from TMEM
-//                (tcgen05 "TS" form; keys 0..63 as soon as that half of P is written, keys
-//                64..127 when the rest is), then S_X = Q_X K_X(j)^T into the same TMEM columns.
-//                While one item's softmax runs, the tensor core works on the other item
-//                (ping-pong). The warp counts each item's valid tiles up front, so its issue
-//                loop reads no global memory;
-//   warp 2       TMEM allocation: S/P_A | S/P_B | O_A | O_B (512 columns for d = 128);
-//   warps 4-7    softmax of item A, warps 8-11 softmax of item B: one thread per query row reads
-//                its 128 logits from TMEM, masks the diagonal block, keeps a running max (O is
-//                rescaled in TMEM, before any P of the tile is published, only when the max
-//                grows by more than 2^8, decided per warp) and running sum, writes P as bf16
-//                back over S in two halves, and at the end normalises O and stores the bf16 row.
-// Because the S/P columns of an item are reused every tile, S_X(j) completing implies the
-// previous PV product of that item completed (MMAs complete in issue order), so O_X is stable
-// whenever its softmax runs.
-// The kept list is read by every role with the same validity rule (0 <= J <= I, strictly
+// One CTA runs one work item: query block I of one head. Its footprint (256 threads, 256 TMEM
+// columns, about 97 KB of shared memory) lets two CTAs share an SM, so the tensor core works on
+// one CTA's tile while the other CTA's softmax runs, and one CTA's set-up and epilogue overlap
+// the other's work. Grid order is longest-first (I descending), by KV-head chunk when K and V
+// exceed L2 (see attn_item). Roles:
+//   warp 0       TMA producer: the Q tile, then V(j-1), K(j) through a two-tile ring, in the
+//                order the MMA warp consumes them;
+//   warp 1       MMA issuer (one thread): O += P(j-1) V(j-1) with P read from TMEM (tcgen05
+//                "TS" form; keys 0..63 as soon as that half of P is written, keys 64..127 when
+//                the rest is), then S = Q K(j)^T into the same TMEM columns. It counts the
+//                item's valid tiles up front, so its issue loop reads no global memory;
+//   warp 2       TMEM allocation: S / P (128 columns) | O (d columns);
+//   warps 4-7    softmax: one thread per query row reads its 128 logits from TMEM, masks the
+//                diagonal block, keeps a running max (O is rescaled in TMEM, before any P of the
+//                tile is published, only when the max grows by more than 2^8, decided per warp)
+//                and running sum, writes P as bf16 back over S in two halves, and at the end
+//                normalises O and stores the bf16 row.
+// Because the S / P columns are reused every tile, S(j) completing implies that the previous
+// P V product completed (MMAs complete in issue order), so O is stable whenever the softmax
+// runs. The kept list is read by every role with the same validity rule (0 <= J <= I, strictly
 // ascending); invalid entries are skipped and flagged in the status word by the producer.
 #include <math.h>
 
@@ -34,8 +32,8 @@ namespace rra {
 
 struct AttnParams {
   int hq, hkv, g, L, nb, batch;
-  int n_pairs;       // batch * ceil(hq / 2)
-  int chunk;         // head pairs per chunk of the launch order (ceil(g / 2) or all)
+  int n_units;       // batch * hq work units (one head each) per query block
+  int chunk;         // heads per chunk of the launch order (one KV head's query heads, or all)
   int64_t tri;
   float scale_log2;
   const int32_t *kept_idx;
@@ -56,12 +54,15 @@ struct ListCursor {
     prev = -1;
     lst = p.kept_idx + static_cast<int64_t>(bh) * p.tri + static_cast<int64_t>(I) * (I + 1) / 2;
     cnt = 0;
+    ahead = -1;
     if (valid) {
+      // both loads issued together: the row has I + 1 >= 1 entries, so lst[0] is in bounds
+      const int first = lst[0];
       cnt = p.kept_cnt[static_cast<int64_t>(bh) * p.nb + I];
       if (cnt < 0) cnt = 0;
       if (cnt > I + 1) cnt = I + 1;
+      ahead = cnt > 0 ? first : -1;
     }
-    ahead = cnt > 0 ? lst[0] : -1;
   }
   // next valid block index, or -1; invalid entries are reported through `status` if non-null
   __device__ int next(uint32_t *status) {
@@ -106,43 +107,42 @@ __device__ int count_valid_warp(const AttnParams &p, int bh, int I, bool valid, 
   return n;
 }
 
-// Launch order: per batch row, chunks of `chunk` head pairs, each chunk's block rows longest
-// first (I descending), the chunk's pairs innermost. With one chunk per batch row this is plain
+// Launch order: per batch row, chunks of `chunk` query heads, each chunk's block rows longest
+// first (I descending), the chunk's heads innermost. With one chunk per batch row this is plain
 // longest-first. With chunks of the query heads of one KV head, the CTAs resident at one time
 // read the K/V tiles of one or two KV heads, which fit in L2 even at long lengths, so a tile kept
 // by several rows or heads is fetched from DRAM about once.
-__device__ __forceinline__ void attn_item(const AttnParams &p, int64_t idx, int &b, int &c,
+__device__ __forceinline__ void attn_item(const AttnParams &p, int64_t idx, int &b, int &h,
                                           int &level) {
-  const int hp = (p.hq + 1) >> 1;
-  const int64_t per_b = static_cast<int64_t>(p.nb) * hp;
+  const int64_t per_b = static_cast<int64_t>(p.nb) * p.hq;
   b = static_cast<int>(idx / per_b);
   const int64_t r = idx - b * per_b;
   const int C = p.chunk;
-  const int nfull = hp / C;
+  const int nfull = p.hq / C;
   const int64_t full = static_cast<int64_t>(nfull) * p.nb * C;
   if (r < full) {
     const int64_t per_chunk = static_cast<int64_t>(p.nb) * C;
     const int k = static_cast<int>(r / per_chunk);
     const int64_t s = r - k * per_chunk;
     level = static_cast<int>(s / C);
-    c = k * C + static_cast<int>(s - static_cast<int64_t>(level) * C);
+    h = k * C + static_cast<int>(s - static_cast<int64_t>(level) * C);
   } else {   // the last, narrower chunk
-    const int crem = hp - nfull * C;
+    const int crem = p.hq - nfull * C;
     const int64_t s = r - full;
     level = static_cast<int>(s / crem);
-    c = nfull * C + static_cast<int>(s - static_cast<int64_t>(level) * crem);
+    h = nfull * C + static_cast<int>(s - static_cast<int64_t>(level) * crem);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(256, 2)
     bs_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   constexpr int NCHUNK = D / 64;
   constexpr uint32_t CHUNK_BYTES = 128 * 128;
   constexpr uint32_t TILE_BYTES = NCHUNK * CHUNK_BYTES;   // 128 rows x D bf16
-  constexpr int NSTAGE = (D == 128) ? 5 : 10;
+  constexpr int NSTAGE = (D == 128) ? 2 : 4;
   constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false);
   constexpr uint32_t IDESC_O = idesc_bf16_f32(128, D, true);
   constexpr float RESCALE_THRESHOLD = 8.0f;               // log2 units
@@ -150,36 +150,28 @@ __global__ void __launch_bounds__(384, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t *sQ = smem;                               // [2] tiles
-  uint8_t *sRing = sQ + 2 * TILE_BYTES;             // [NSTAGE] tiles
+  uint8_t *sQ = smem;
+  uint8_t *sRing = sQ + TILE_BYTES;                 // [NSTAGE] tiles
   uint64_t *bars = reinterpret_cast<uint64_t *>(sRing + NSTAGE * TILE_BYTES);
   uint64_t *q_full = bars + 0;
   uint64_t *kv_full = bars + 1;                     // [NSTAGE]
   uint64_t *kv_empty = kv_full + NSTAGE;            // [NSTAGE]
-  uint64_t *s_full = kv_empty + NSTAGE;             // [2]
-  uint64_t *p_full = s_full + 2;                    // [2]
-  uint64_t *p_half = p_full + 2;                    // [2] P of keys 0..63 written
-  uint64_t *o_final = p_half + 2;                   // [2]
-  uint64_t *drain = o_final + 2;
+  uint64_t *s_full = kv_empty + NSTAGE;
+  uint64_t *p_full = s_full + 1;
+  uint64_t *p_half = p_full + 1;                    // P of keys 0..63 written
+  uint64_t *o_final = p_half + 1;
+  uint64_t *drain = o_final + 1;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
   volatile int *s_flag = reinterpret_cast<volatile int *>(s_tmem + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  int b, c, level;
-  attn_item(p, blockIdx.x, b, c, level);
+  int b, h, level;
+  attn_item(p, blockIdx.x, b, h, level);
   const int I = p.nb - 1 - level;
-  const int h0 = 2 * c;
-  int bh[2], kvrow[2];
-  bool valid[2];
-#pragma unroll
-  for (int x = 0; x < 2; ++x) {
-    const int h = h0 + x;
-    valid[x] = h < p.hq;
-    bh[x] = b * p.hq + (valid[x] ? h : h0);
-    kvrow[x] = (b * p.hkv + (valid[x] ? h : h0) / p.g) * p.L;
-  }
+  const int bh = b * p.hq + h;
+  const int kvrow = (b * p.hkv + h / p.g) * p.L;
 
   if (cta_grid_timed_out(p.status, s_flag)) return;   // the same answer for every thread
   if (threadIdx.x == 0) {
@@ -188,18 +180,16 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 128);
-      mbar_init(&p_half[x], 128);
-      mbar_init(&o_final[x], 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(p_half, 128);
+    mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *s_abort = 0;
     fence_mbar_init();
   }
   if (warp == 2) {
-    tmem_alloc(s_tmem, 512);
+    tmem_alloc(s_tmem, 256);
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
@@ -211,9 +201,8 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  // columns: S/P of item x at 128*x, O of item x at 256 + D*x
-  auto tm_s = [&](int x) { return tmem + 128u * x; };
-  auto tm_o = [&](int x) { return tmem + 256u + static_cast<uint32_t>(D) * x; };
+  const uint32_t tm_s = tmem;          // S / P: columns 0..127
+  const uint32_t tm_o = tmem + 128u;   // O: columns 128..128+D
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -236,115 +225,93 @@ __global__ void __launch_bounds__(384, 1)
         }
         return true;
       };
-      ListCursor cur[2];
-      int J[2], pendV[2] = {-1, -1};
-      for (int x = 0; x < 2; ++x) {
-        cur[x].init(p, bh[x], I, valid[x]);
-        J[x] = cur[x].next(p.status);
-      }
-      const bool q_any = J[0] >= 0 || J[1] >= 0;
-      if (q_any) {
-        mbar_arrive_expect_tx(q_full, TILE_BYTES * ((J[0] >= 0) + (J[1] >= 0)));
-        for (int x = 0; x < 2; ++x)
-          if (J[x] >= 0)
-            for (int c = 0; c < NCHUNK; ++c)
-              tma_load_2d(sQ + x * TILE_BYTES + c * CHUNK_BYTES, &tm_q, q_full, c * 64,
-                          bh[x] * p.L + I * 128);
-      }
-      while (ok) {
-        bool any = false;
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (pendV[x] >= 0) {
-            ok = load(&tm_v, kvrow[x] + pendV[x] * 128);
-            pendV[x] = -1;
-            any = true;
-          }
-          if (ok && J[x] >= 0) {
-            ok = load(&tm_k, kvrow[x] + J[x] * 128);
-            pendV[x] = J[x];
-            J[x] = cur[x].next(p.status);
-            any = true;
-          }
+      // the Q tile first: its load overlaps the reads of the kept list (a row with no valid
+      // entry, rare, loads it for nothing)
+      mbar_arrive_expect_tx(q_full, TILE_BYTES);
+      for (int c = 0; c < NCHUNK; ++c)
+        tma_load_2d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, bh * p.L + I * 128);
+      ListCursor cur;
+      cur.init(p, bh, I, true);
+      int J = cur.next(p.status), pendV = -1;
+      // the MMA warp's order: V(j - 1) for P(j - 1) V(j - 1), then K(j) for S(j)
+      while (ok && (pendV >= 0 || J >= 0)) {
+        if (pendV >= 0) {
+          ok = load(&tm_v, kvrow + pendV * 128);
+          pendV = -1;
         }
-        if (!any) break;
+        if (ok && J >= 0) {
+          ok = load(&tm_k, kvrow + J * 128);
+          pendV = J;
+          J = cur.next(p.status);
+        }
       }
       // Let every copy already issued land before the CTA exits (without an abort these
       // phases have completed already: the MMA warp consumed them).
-      if (q_any) mbar_wait_drain(q_full, 0);
+      mbar_wait_drain(q_full, 0);
       for (int s = 0; s < NSTAGE; ++s)
         if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Tile counts first (whole warp), so the issue loop itself touches no global memory.
-    int n[2];
-#pragma unroll
-    for (int x = 0; x < 2; ++x) n[x] = count_valid_warp(p, bh[x], I, valid[x], lane);
+    const int n = count_valid_warp(p, bh, I, true, lane);
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      if (n[0] + n[1] > 0) ok = mbar_wait(q_full, 0, s_abort, p.status, p.wait_ns);
-      // descriptors: base of each operand; per-MMA offsets are added in 16-byte units
+      if (n > 0) ok = mbar_wait(q_full, 0, s_abort, p.status, p.wait_ns);
       const uint32_t ring_base = smem_u32(sRing);
-      const uint64_t q_desc[2] = {sdesc_kmajor_sw128(smem_u32(sQ)),
-                                  sdesc_kmajor_sw128(smem_u32(sQ) + TILE_BYTES)};
+      const uint64_t q_desc = sdesc_kmajor_sw128(smem_u32(sQ));
       const uint64_t k_desc0 = sdesc_kmajor_sw128(ring_base);
       const uint64_t v_desc0 = sdesc_mnmajor_sw128(ring_base, CHUNK_BYTES);
-      const int steps = max(n[0], n[1]);
-      for (int j = 0; j <= steps && ok; ++j) {
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          if (j >= 1 && j <= n[x]) {
-            // O_x += P_x(j-1) V_x(j-1); P sits in the S columns of item x. Keys 0..63 go in
-            // as soon as their half of P is written, while the softmax finishes keys 64..127.
-            if (!mbar_wait(&p_half[x], (j - 1) & 1, s_abort, p.status, p.wait_ns) ||
-                !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t vd = v_desc0 + ((stage * TILE_BYTES) >> 4);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
-                          (j > 1 || kk > 0) ? 1u : 0u);
-            if (!mbar_wait(&p_full[x], (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 4; kk < 8; ++kk)
-              mma_bf16_ts(tm_o(x), tm_s(x) + kk * 8, vd + kk * (2048 >> 4), IDESC_O, 1u);
-            mma_commit(&kv_empty[stage]);
-            if (j == n[x]) mma_commit(&o_final[x]);
-            if (++stage == NSTAGE) {
-              stage = 0;
-              phase ^= 1;
-            }
+      for (int j = 0; j <= n && ok; ++j) {
+        if (j >= 1) {
+          // O += P(j-1) V(j-1): keys 0..63 as soon as their half of P is written
+          if (!mbar_wait(p_half, (j - 1) & 1, s_abort, p.status, p.wait_ns) ||
+              !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
+            ok = false;
+            break;
           }
-          if (j < n[x]) {
-            // S_x = Q_x K_x(j)^T into the same TMEM columns
-            if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t kd = k_desc0 + ((stage * TILE_BYTES) >> 4);
+          tc_fence_after();
+          const uint64_t vd = v_desc0 + ((stage * TILE_BYTES) >> 4);
 #pragma unroll
-            for (int c = 0; c < NCHUNK; ++c)
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
+                        (j > 1 || kk > 0) ? 1u : 0u);
+          if (!mbar_wait(p_full, (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t off = (c * CHUNK_BYTES + kk * 32) >> 4;
-                mma_bf16_ss(tm_s(x), q_desc[x] + off, kd + off, IDESC_S, (c | kk) != 0);
-              }
-            mma_commit(&kv_empty[stage]);
-            mma_commit(&s_full[x]);
-            if (++stage == NSTAGE) {
-              stage = 0;
-              phase ^= 1;
+          for (int kk = 4; kk < 8; ++kk)
+            mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O, 1u);
+          mma_commit(&kv_empty[stage]);
+          if (j == n) mma_commit(o_final);
+          if (++stage == NSTAGE) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (j < n) {
+          // S = Q K(j)^T into the S / P columns
+          if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t kd = k_desc0 + ((stage * TILE_BYTES) >> 4);
+#pragma unroll
+          for (int c = 0; c < NCHUNK; ++c)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint32_t off = (c * CHUNK_BYTES + kk * 32) >> 4;
+              mma_bf16_ss(tm_s, q_desc + off, kd + off, IDESC_S, (c | kk) != 0);
             }
+          mma_commit(&kv_empty[stage]);
+          mma_commit(s_full);
+          if (++stage == NSTAGE) {
+            stage = 0;
+            phase ^= 1;
           }
         }
       }
@@ -353,12 +320,11 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int x = (warp - 4) >> 2;       // item
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const uint32_t s_cols = tm_s(x) + lane_off;
-    const uint32_t o_cols = tm_o(x) + lane_off;
+    const uint32_t s_cols = tm_s + lane_off;
+    const uint32_t o_cols = tm_o + lane_off;
     const float NEG_INF = -INFINITY;
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -366,10 +332,10 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t lsum[4] = {0, 0, 0, 0};
     bool dead = false;
     ListCursor cur;
-    cur.init(p, bh[x], I, valid[x]);
+    cur.init(p, bh, I, true);
     int t = 0;
     for (int J = cur.next(nullptr); J >= 0; J = cur.next(nullptr), ++t) {
-      if (!mbar_wait_warp(&s_full[x], t & 1, s_abort, p.status, p.wait_ns)) {
+      if (!mbar_wait_warp(s_full, t & 1, s_abort, p.status, p.wait_ns)) {
         dead = true;
         break;
       }
@@ -378,15 +344,15 @@ __global__ void __launch_bounds__(384, 1)
       // pass 1: row max over the 128 logits, 64 columns at a time
       float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      for (int hh = 0; hh < 2; ++hh) {
         float u[64];
-        tmem_ld32(s_cols + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tmem_ld32(s_cols + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_ld32(s_cols + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(s_cols + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
         tmem_ld_wait();
         if (diag) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (h * 64 + c > r) u[c] = NEG_INF;
+            if (hh * 64 + c > r) u[c] = NEG_INF;
         }
 #pragma unroll
         for (int c = 0; c < 64; c += 8) {
@@ -406,14 +372,13 @@ __global__ void __launch_bounds__(384, 1)
         alpha = fast_exp2(m_run - m_new);
         m_run = m_new;
         rescale = true;
-        // the sum so far was taken against the old max; this tile's terms are added below
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
         for (int c = 0; c < 4; ++c) lsum[c] = fmul2(lsum[c], a2);
       }
       if (rescale) {
-        // O_x is final for the previous tile (S_x(t) completing implies it). It is rescaled
-        // before any P of this tile is published, since the PV product starts on the first half.
+        // O is final for the previous tile (S(t) completing implies it); rescaled before any
+        // P of this tile is published
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -424,20 +389,18 @@ __global__ void __launch_bounds__(384, 1)
           tmem_st32(o_cols + c * 32, o);
         }
       }
-      // pass 2: P = 2^(u*scale_log2 - m) in bf16, written over S. Keys 0..63 are re-read and
-      // packed into columns 0..31 and published (p_half) before keys 64..127 are re-read: their
-      // packed P lands in columns 32..63, whose logits (keys 32..63) are consumed by then.
+      // pass 2: P = 2^(u * scale_log2 - m) in bf16, written over S in two halves
       const uint64_t negm = f2_pack(-m_run, -m_run);
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
+      for (int hh = 0; hh < 2; ++hh) {
         float u[64];
-        tmem_ld32(s_cols + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tmem_ld32(s_cols + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+        tmem_ld32(s_cols + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+        tmem_ld32(s_cols + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
         tmem_ld_wait();
         if (diag) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (h * 64 + c > r) u[c] = NEG_INF;
+            if (hh * 64 + c > r) u[c] = NEG_INF;
         }
         uint32_t pk[32];
 #pragma unroll
@@ -448,61 +411,59 @@ __global__ void __launch_bounds__(384, 1)
           lsum[q & 3] = fadd2(lsum[q & 3], f2_pack(p0, p1));
           pk[q] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(s_cols + h * 32, pk);
+        tmem_st32(s_cols + hh * 32, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(h == 0 ? &p_half[x] : &p_full[x]);
+        mbar_arrive(hh == 0 ? p_half : p_full);
       }
     }
-    if (valid[x]) {
-      __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh[x]) * p.L + I * 128 + r) * D;
-      if (!dead && t > 0 && mbar_wait_warp(&o_final[x], 0, s_abort, p.status, p.wait_ns)) {
-        tc_fence_after();
-        const uint64_t s01 = fadd2(lsum[0], lsum[1]), s23 = fadd2(lsum[2], lsum[3]);
-        const uint64_t s4 = fadd2(s01, s23);
-        const float inv = 1.f / (f2_lo(s4) + f2_hi(s4));
+    __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh) * p.L + I * 128 + r) * D;
+    if (!dead && t > 0 && mbar_wait_warp(o_final, 0, s_abort, p.status, p.wait_ns)) {
+      tc_fence_after();
+      const uint64_t s01 = fadd2(lsum[0], lsum[1]), s23 = fadd2(lsum[2], lsum[3]);
+      const uint64_t s4 = fadd2(s01, s23);
+      const float inv = 1.f / (f2_lo(s4) + f2_hi(s4));
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_cols + c * 32, o);
-          tmem_ld_wait();
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(o_cols + c * 32, o);
+        tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 32; q += 8) {
-            uint4 v;
-            v.x = pack_bf16x2(__uint_as_float(o[q]) * inv, __uint_as_float(o[q + 1]) * inv);
-            v.y = pack_bf16x2(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv);
-            v.z = pack_bf16x2(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv);
-            v.w = pack_bf16x2(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv);
-            *reinterpret_cast<uint4 *>(orow + c * 32 + q) = v;
-          }
+        for (int q = 0; q < 32; q += 8) {
+          uint4 v;
+          v.x = pack_bf16x2(__uint_as_float(o[q]) * inv, __uint_as_float(o[q + 1]) * inv);
+          v.y = pack_bf16x2(__uint_as_float(o[q + 2]) * inv, __uint_as_float(o[q + 3]) * inv);
+          v.z = pack_bf16x2(__uint_as_float(o[q + 4]) * inv, __uint_as_float(o[q + 5]) * inv);
+          v.w = pack_bf16x2(__uint_as_float(o[q + 6]) * inv, __uint_as_float(o[q + 7]) * inv);
+          *reinterpret_cast<uint4 *>(orow + c * 32 + q) = v;
         }
-      } else if (!dead && t == 0) {
-#pragma unroll
-        for (int c = 0; c < D; c += 8)
-          *reinterpret_cast<uint4 *>(orow + c) = make_uint4(0, 0, 0, 0);
       }
+    } else if (!dead && t == 0) {
+#pragma unroll
+      for (int c = 0; c < D; c += 8)
+        *reinterpret_cast<uint4 *>(orow + c) = make_uint4(0, 0, 0, 0);
     }
     tc_fence_before();
   }
   __syncthreads();
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
 }
 
 template <int D>
 static cudaError_t launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk,
-                                 const CUtensorMap &mv, const AttnParams &ap, int64_t grid,
-                                 cudaStream_t stream) {
+                                  const CUtensorMap &mv, const AttnParams &ap, int64_t grid,
+                                  cudaStream_t stream) {
   constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
-  constexpr int NSTAGE = (D == 128) ? 5 : 10;
-  const size_t smem = 1024 + TILE * (2 + NSTAGE) + (2 * NSTAGE + 10) * 8 + 16;
+  constexpr int NSTAGE = (D == 128) ? 2 : 4;
+  const size_t smem = 1024 + TILE * (1 + NSTAGE) + (2 * NSTAGE + 6) * 8 + 16;
   auto kern = bs_attn_fwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(grid), 384, smem, stream>>>(mq, mk, mv, ap);
+  kern<<<static_cast<unsigned>(grid), 256, smem, stream>>>(mq, mk, mv, ap);
   return cudaGetLastError();
 }
 
@@ -548,11 +509,11 @@ cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, 
   ap.L = g.L;
   ap.nb = g.nb;
   ap.batch = g.b;
-  ap.n_pairs = g.b * ((g.hq + 1) / 2);
+  ap.n_units = g.b * g.hq;
   // KV-head chunks only when K and V of all heads are well beyond L2: then the chunked order
   // keeps re-read tiles in L2. Below that the plain longest-first order balances the tail better.
   const int64_t kv_bytes = static_cast<int64_t>(g.b) * g.hkv * g.L * g.d * 2 * 2;
-  ap.chunk = kv_bytes > 2 * l2_bytes() ? (g.g + 1) / 2 : (g.hq + 1) / 2;
+  ap.chunk = kv_bytes > 2 * l2_bytes() ? g.g : g.hq;
   ap.tri = g.tri;
   ap.scale_log2 = g.scale * 1.4426950408889634f;
   ap.kept_idx = kept_idx;
@@ -560,7 +521,7 @@ cudaError_t launch_sparse_attn(const Geometry &g, const void *q, const void *k, 
   ap.out = static_cast<__nv_bfloat16 *>(out);
   ap.status = status;
   ap.wait_ns = wait_limit_ns();
-  const int64_t grid = static_cast<int64_t>(ap.n_pairs) * g.nb;
+  const int64_t grid = static_cast<int64_t>(ap.n_units) * g.nb;
   if (g.d == 128) return launch_attn_t<128>(mq, mk, mv, ap, grid, stream);
   if (g.d == 64) return launch_attn_t<64>(mq, mk, mv, ap, grid, stream);
   return cudaErrorInvalidValue;
