@@ -734,6 +734,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama128k", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--stride", type=int, default=None, help="override the workload's S")
+    ap.add_argument("--tau", type=float, default=None, help="override the workload's tau")
+    ap.add_argument("--seqlen", type=int, default=None, help="override the workload's L")
+    ap.add_argument("--shift", type=int, default=None, help="override the round-robin shift")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=None,
                     help="seeded query blocks of oracle attention in the CPU baseline "
@@ -754,6 +758,10 @@ def main(argv=None):
     if args.study == "search":
         return run_search_study(args)
     w = wl.WORKLOADS[args.workload]
+    over = {k: getattr(args, k) for k in ("stride", "tau", "seqlen", "shift")
+            if getattr(args, k) is not None}
+    if over:   # the same recipe and seed at other settings (e.g. the 32K sweep points)
+        w = w.with_(**over)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

@@ -53,3 +53,13 @@ def test_head_density_and_attention_flops():
     assert bench.head_density(cnt)["max"] == 1.0
     useful, _, n = bench.attention_flops(idx, cnt, 128, 64)
     assert n == 10 and useful == 4.0 * 64 * (128 * 128 * 6 + 128 * 129 / 2 * 4)
+
+
+def test_workload_overrides_reach_the_config():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--stride", "16", "--tau", "0.95", "--steps", "1",
+                        "--warmup", "0"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["config"]["stride"] == 16 and d["config"]["tau"] == 0.95
+    assert "S16" in d["config"]["workload"] and "tau0.95" in d["config"]["workload"]
