@@ -190,18 +190,16 @@ def mass_rows(full: dict, nb: int) -> dict:
 
 # ------------------------------------------------------------------ parity report
 # Every parity check appends one record here; tests/conftest.py prints them at the end of the
-# session (so the boundary-excused counts appear in `pytest -q` output), and if the directory
-# named by RRA_PARITY_REPORT (default: the repository's gpurun_out/, when it exists) is present
-# each record is also appended to parity_report.jsonl there.
+# session (so the boundary-excused counts appear in `pytest -q` output). If RRA_PARITY_REPORT
+# names an existing directory, each record is also appended to parity_report.jsonl there.
 RECORDS: list = []
 
 
 def record(label: str, **fields) -> dict:
     rec = {"label": label, **fields, "when": time.strftime("%Y-%m-%dT%H:%M:%S")}
     RECORDS.append(rec)
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    out_dir = os.environ.get("RRA_PARITY_REPORT", os.path.join(root, "gpurun_out"))
-    if os.path.isdir(out_dir):
+    out_dir = os.environ.get("RRA_PARITY_REPORT")
+    if out_dir and os.path.isdir(out_dir):
         with open(os.path.join(out_dir, "parity_report.jsonl"), "a") as f:
             f.write(json.dumps(rec) + "\n")
     return rec
