@@ -17,8 +17,8 @@
 //   warps 4-7    softmax: one thread per query row reads its 128 logits from TMEM, masks the
 //                diagonal block, keeps a running max (O is rescaled in TMEM, before any P of the
 //                tile is published, only when the max grows by more than 2^8, decided per warp)
-//                and running sum, writes P as bf16 back over S in two halves, and at the end
-//                normalises O and stores the bf16 row.
+//                and running sum of the bf16-rounded weights, writes P as bf16 back over S in
+//                two halves, and at the end normalises O and stores the bf16 row.
 // Because the S / P columns are reused every tile, S(j) completing implies that the previous
 // P V product completed (MMAs complete in issue order), so O is stable whenever the softmax
 // runs. The kept list is read by every role with the same validity rule (0 <= J <= I, strictly
@@ -406,10 +406,11 @@ __global__ void __launch_bounds__(256, 2)
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
           const uint64_t xy = ffma2(f2_pack(u[2 * q], u[2 * q + 1]), sl2x2, negm);
-          const float p0 = fast_exp2(f2_lo(xy));
-          const float p1 = fast_exp2(f2_hi(xy));
-          lsum[q & 3] = fadd2(lsum[q & 3], f2_pack(p0, p1));
-          pk[q] = pack_bf16x2(p0, p1);
+          pk[q] = pack_bf16x2(fast_exp2(f2_lo(xy)), fast_exp2(f2_hi(xy)));
+          // the row sum takes the bf16 weights that P V uses, so O / l stays a convex
+          // combination of the V rows (one dominant weight is no longer off by its rounding)
+          lsum[q & 3] = fadd2(lsum[q & 3], f2_pack(__uint_as_float(pk[q] << 16),
+                                                   __uint_as_float(pk[q] & 0xffff0000u)));
         }
         tmem_st32(s_cols + hh * 32, pk);
         tmem_st_wait();

@@ -56,3 +56,60 @@ def masses_full(q_bits, k_bits, batch, heads_q, heads_kv, seqlen, block, stride,
             else:
                 os.environ[v] = old
     return dict(zip(keys, res))
+
+
+def head_attention_errors(args):
+    """Oracle attention of every query block of one (batch, head) on the GPU's kept lists,
+    compared with the GPU's output rows: (max |gpu - ref|, sum (gpu - ref)^2, sum ref^2)."""
+    q_bits, k_bits, v_bits, gpu_out, idx, cnt, block, scale = args
+    q = wl.bf16_bits_to_f64(q_bits)
+    k = wl.bf16_bits_to_f64(k_bits)
+    v = wl.bf16_bits_to_f64(v_bits)
+    nb = q.shape[0] // block
+    max_abs, sq_diff, sq_ref = 0.0, 0.0, 0.0
+    for I in range(nb):
+        off = orc.tri_offset(I)
+        ref = orc.attention_block(q, k, v, I, idx[off:off + int(cnt[I])], block, scale)
+        diff = gpu_out[I * block:(I + 1) * block].astype(np.float64) - ref
+        max_abs = max(max_abs, float(np.abs(diff).max()))
+        sq_diff += float(np.sum(diff * diff))
+        sq_ref += float(np.sum(ref * ref))
+    return max_abs, sq_diff, sq_ref
+
+
+def attention_errors_full(q_bits, k_bits, v_bits, gpu_out, idx, cnt, heads_q, heads_kv, block,
+                          scale, workers=None):
+    """Every output row of every (batch, head) against the oracle, one head per task on a pool
+    of spawned processes: (max-abs error, relative RMS error, rows compared). gpu_out is the GPU
+    output as a float32 array [b, Hq, L, d]; idx / cnt are the GPU's kept lists."""
+    b = gpu_out.shape[0]
+    keys = [(bi, h) for bi in range(b) for h in range(heads_q)]
+
+    def task(bi, h):
+        kv = orc.kv_head(h, heads_q, heads_kv)
+        return (np.ascontiguousarray(q_bits[bi, h]), np.ascontiguousarray(k_bits[bi, kv]),
+                np.ascontiguousarray(v_bits[bi, kv]), np.ascontiguousarray(gpu_out[bi, h]),
+                np.ascontiguousarray(idx[bi, h]), np.ascontiguousarray(cnt[bi, h]), block, scale)
+
+    if workers is None:
+        workers = max(1, min(len(keys), len(os.sched_getaffinity(0))))
+    if workers == 1:
+        res = [head_attention_errors(task(bi, h)) for bi, h in keys]
+    else:
+        names = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+        saved = {v: os.environ.get(v) for v in names}
+        for v in names:
+            os.environ[v] = "1"
+        try:
+            ctx = multiprocessing.get_context("spawn")
+            with concurrent.futures.ProcessPoolExecutor(workers, mp_context=ctx) as ex:
+                res = list(ex.map(head_attention_errors, (task(bi, h) for bi, h in keys)))
+        finally:
+            for v, old in saved.items():
+                if old is None:
+                    os.environ.pop(v, None)
+                else:
+                    os.environ[v] = old
+    max_abs = max(r[0] for r in res)
+    rel_rms = float(np.sqrt(sum(r[1] for r in res) / max(sum(r[2] for r in res), 1e-300)))
+    return max_abs, rel_rms, len(keys) * (gpu_out.shape[2] // block)

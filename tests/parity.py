@@ -250,13 +250,17 @@ def long_check(w, p, bits, gpu, label, attn_rows, seed, mass_heads=None):
     rows = mass_rows(full, nb)
     mism, exc, n = compare_select_rows(gpu, rows, w.tau)
     assert not mism, f"{label}: kept-list mismatches outside the boundary rule: {mism[:5]}"
-    qc, kc, vc = HeadCache(qb), HeadCache(kb), HeadCache(vb)
     if attn_rows == "all":
-        arows = [(b, h, I) for b in range(w.batch) for h in range(w.heads_q) for I in range(nb)]
+        import oracle_pool
+        ma, rr, n_attn = oracle_pool.attention_errors_full(
+            qb, kb, vb, gpu["out"], gpu["idx"], gpu["cnt"], p.heads_q, p.heads_kv, p.block,
+            resolved_scale(p))
+        arows = range(n_attn)
     else:
+        qc, kc, vc = HeadCache(qb), HeadCache(kb), HeadCache(vb)
         arows = sample_rows(p, attn_rows, seed)
-    ref = oracle_attention_rows(qc, kc, vc, p, gpu["idx"], gpu["cnt"], arows)
-    ma, rr = attention_rows_errors(gpu["out"], ref)
+        ref = oracle_attention_rows(qc, kc, vc, p, gpu["idx"], gpu["cnt"], arows)
+        ma, rr = attention_rows_errors(gpu["out"], ref)
     assert ma <= ATTN_MAX_ABS and rr <= ATTN_REL_RMS, f"{label}: attn {ma} {rr}"
     dens = gpu["cnt"].sum(dtype=np.int64) / (w.batch * w.heads_q * orc.tri_offset(nb))
     record(label, mass_rows=n, mass_max_err=merr, list_rows=n,
