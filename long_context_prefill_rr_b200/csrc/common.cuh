@@ -308,6 +308,15 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
+// a += low bf16 of w, b += high bf16 of w: mixed-precision adds (bf16 operand, f32 sum), so
+// summing packed bf16 values costs one instruction per value
+__device__ __forceinline__ void add_bf16x2_to_f32(float &a, float &b, uint32_t w) {
+  unsigned short lo, hi;
+  asm("mov.b32 {%0, %1}, %2;" : "=h"(lo), "=h"(hi) : "r"(w));
+  asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(a) : "h"(lo));
+  asm("add.rn.f32.bf16 %0, %1, %0;" : "+f"(b) : "h"(hi));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);   // .x = lo (low 16 bits), .y = hi
   return *reinterpret_cast<uint32_t *>(&v);

@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(256, 2)
     const float sl2 = p.scale_log2;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_run = NEG_INF;
-    uint64_t lsum[4] = {0, 0, 0, 0};
+    float lsum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     bool dead = false;
     ListCursor cur;
     cur.init(p, bh, I, true);
@@ -372,9 +372,8 @@ __global__ void __launch_bounds__(256, 2)
         alpha = fast_exp2(m_run - m_new);
         m_run = m_new;
         rescale = true;
-        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) lsum[c] = fmul2(lsum[c], a2);
+        for (int c = 0; c < 8; ++c) lsum[c] *= alpha;
       }
       if (rescale) {
         // O is final for the previous tile (S(t) completing implies it); rescaled before any
@@ -409,8 +408,7 @@ __global__ void __launch_bounds__(256, 2)
           pk[q] = pack_bf16x2(fast_exp2(f2_lo(xy)), fast_exp2(f2_hi(xy)));
           // the row sum takes the bf16 weights that P V uses, so O / l stays a convex
           // combination of the V rows (one dominant weight is no longer off by its rounding)
-          lsum[q & 3] = fadd2(lsum[q & 3], f2_pack(__uint_as_float(pk[q] << 16),
-                                                   __uint_as_float(pk[q] & 0xffff0000u)));
+          add_bf16x2_to_f32(lsum[(2 * q) & 7], lsum[(2 * q + 1) & 7], pk[q]);
         }
         tmem_st32(s_cols + hh * 32, pk);
         tmem_st_wait();
@@ -421,9 +419,8 @@ __global__ void __launch_bounds__(256, 2)
     __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh) * p.L + I * 128 + r) * D;
     if (!dead && t > 0 && mbar_wait_warp(o_final, 0, s_abort, p.status, p.wait_ns)) {
       tc_fence_after();
-      const uint64_t s01 = fadd2(lsum[0], lsum[1]), s23 = fadd2(lsum[2], lsum[3]);
-      const uint64_t s4 = fadd2(s01, s23);
-      const float inv = 1.f / (f2_lo(s4) + f2_hi(s4));
+      const float inv = 1.f / (((lsum[0] + lsum[1]) + (lsum[2] + lsum[3])) +
+                               ((lsum[4] + lsum[5]) + (lsum[6] + lsum[7])));
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
