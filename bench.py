@@ -725,7 +725,7 @@ def run_search_study(args):
 
 
 # bump when the attention kernel changes, so stale ncu traffic is not reported
-KERNEL_REV = "attn-v6-rsum"
+KERNEL_REV = "attn-v7-nreg"
 
 
 def main(argv=None):

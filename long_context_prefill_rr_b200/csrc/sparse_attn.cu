@@ -19,6 +19,8 @@
 //                tile is published, only when the max grows by more than 2^8, decided per warp)
 //                and running sum of the bf16-rounded weights, writes P as bf16 back over S in
 //                two halves, and at the end normalises O and stores the bf16 row.
+// The first warpgroup (warps 0-3) runs with 96 registers a thread and the softmax warpgroup
+// with 160 (setmaxnreg), out of the 128 a thread the CTA is launched with.
 // Because the S / P columns are reused every tile, S(j) completing implies that the previous
 // P V product completed (MMAs complete in issue order), so O is stable whenever the softmax
 // runs. The kept list is read by every role with the same validity rule (0 <= J <= I, strictly
@@ -204,121 +206,128 @@ __global__ void __launch_bounds__(256, 2)
   const uint32_t tm_s = tmem;          // S / P: columns 0..127
   const uint32_t tm_o = tmem + 128u;   // O: columns 128..128+D
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued[NSTAGE];
-      for (int s = 0; s < NSTAGE; ++s) issued[s] = 0;
-      bool ok = true;
-      auto load = [&](const CUtensorMap *map, int row) -> bool {
-        if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status, p.wait_ns)) return false;
-        mbar_arrive_expect_tx(&kv_full[stage], TILE_BYTES);
-        uint8_t *dst = sRing + stage * TILE_BYTES;
-        for (int c = 0; c < NCHUNK; ++c)
-          tma_load_2d(dst + c * CHUNK_BYTES, map, &kv_full[stage], c * 64, row);
-        ++issued[stage];
-        if (++stage == NSTAGE) {
-          stage = 0;
-          phase ^= 1;
-        }
-        return true;
-      };
-      // the Q tile first: its load overlaps the reads of the kept list (a row with no valid
-      // entry, rare, loads it for nothing)
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      for (int c = 0; c < NCHUNK; ++c)
-        tma_load_2d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, bh * p.L + I * 128);
-      ListCursor cur;
-      cur.init(p, bh, I, true);
-      int J = cur.next(p.status), pendV = -1;
-      // the MMA warp's order: V(j - 1) for P(j - 1) V(j - 1), then K(j) for S(j)
-      while (ok && (pendV >= 0 || J >= 0)) {
-        if (pendV >= 0) {
-          ok = load(&tm_v, kvrow + pendV * 128);
-          pendV = -1;
-        }
-        if (ok && J >= 0) {
-          ok = load(&tm_k, kvrow + J * 128);
-          pendV = J;
-          J = cur.next(p.status);
-        }
-      }
-      // Let every copy already issued land before the CTA exits (without an abort these
-      // phases have completed already: the MMA warp consumed them).
-      mbar_wait_drain(q_full, 0);
-      for (int s = 0; s < NSTAGE; ++s)
-        if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    const int n = count_valid_warp(p, bh, I, true, lane);
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      if (n > 0) ok = mbar_wait(q_full, 0, s_abort, p.status, p.wait_ns);
-      const uint32_t ring_base = smem_u32(sRing);
-      const uint64_t q_desc = sdesc_kmajor_sw128(smem_u32(sQ));
-      const uint64_t k_desc0 = sdesc_kmajor_sw128(ring_base);
-      const uint64_t v_desc0 = sdesc_mnmajor_sw128(ring_base, CHUNK_BYTES);
-      for (int j = 0; j <= n && ok; ++j) {
-        if (j >= 1) {
-          // O += P(j-1) V(j-1): keys 0..63 as soon as their half of P is written
-          if (!mbar_wait(p_half, (j - 1) & 1, s_abort, p.status, p.wait_ns) ||
-              !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t vd = v_desc0 + ((stage * TILE_BYTES) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
-                        (j > 1 || kk > 0) ? 1u : 0u);
-          if (!mbar_wait(p_full, (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 4; kk < 8; ++kk)
-            mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O, 1u);
-          mma_commit(&kv_empty[stage]);
-          if (j == n) mma_commit(o_final);
-          if (++stage == NSTAGE) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (j < n) {
-          // S = Q K(j)^T into the S / P columns
-          if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t kd = k_desc0 + ((stage * TILE_BYTES) >> 4);
-#pragma unroll
+  if (warp < 4) {
+    // Register split between the warpgroups: the producer / MMA / allocator warpgroup gives up
+    // registers so that the softmax warpgroup can keep its row slice and more exponentials in
+    // flight (96 + 160 = 2 x the 128 the CTA was launched with).
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 96;\n" ::: "memory");
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int issued[NSTAGE];
+        for (int s = 0; s < NSTAGE; ++s) issued[s] = 0;
+        bool ok = true;
+        auto load = [&](const CUtensorMap *map, int row) -> bool {
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1, s_abort, p.status, p.wait_ns)) return false;
+          mbar_arrive_expect_tx(&kv_full[stage], TILE_BYTES);
+          uint8_t *dst = sRing + stage * TILE_BYTES;
           for (int c = 0; c < NCHUNK; ++c)
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint32_t off = (c * CHUNK_BYTES + kk * 32) >> 4;
-              mma_bf16_ss(tm_s, q_desc + off, kd + off, IDESC_S, (c | kk) != 0);
-            }
-          mma_commit(&kv_empty[stage]);
-          mma_commit(s_full);
+            tma_load_2d(dst + c * CHUNK_BYTES, map, &kv_full[stage], c * 64, row);
+          ++issued[stage];
           if (++stage == NSTAGE) {
             stage = 0;
             phase ^= 1;
           }
+          return true;
+        };
+        // the Q tile first: its load overlaps the reads of the kept list (a row with no valid
+        // entry, rare, loads it for nothing)
+        mbar_arrive_expect_tx(q_full, TILE_BYTES);
+        for (int c = 0; c < NCHUNK; ++c)
+          tma_load_2d(sQ + c * CHUNK_BYTES, &tm_q, q_full, c * 64, bh * p.L + I * 128);
+        ListCursor cur;
+        cur.init(p, bh, I, true);
+        int J = cur.next(p.status), pendV = -1;
+        // the MMA warp's order: V(j - 1) for P(j - 1) V(j - 1), then K(j) for S(j)
+        while (ok && (pendV >= 0 || J >= 0)) {
+          if (pendV >= 0) {
+            ok = load(&tm_v, kvrow + pendV * 128);
+            pendV = -1;
+          }
+          if (ok && J >= 0) {
+            ok = load(&tm_k, kvrow + J * 128);
+            pendV = J;
+            J = cur.next(p.status);
+          }
         }
+        // Let every copy already issued land before the CTA exits (without an abort these
+        // phases have completed already: the MMA warp consumed them).
+        mbar_wait_drain(q_full, 0);
+        for (int s = 0; s < NSTAGE; ++s)
+          if (issued[s] > 0) mbar_wait_drain(&kv_full[s], (issued[s] - 1) & 1);
       }
-      mma_commit(drain);
-      mbar_wait_drain(drain, 0);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      const int n = count_valid_warp(p, bh, I, true, lane);
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        if (n > 0) ok = mbar_wait(q_full, 0, s_abort, p.status, p.wait_ns);
+        const uint32_t ring_base = smem_u32(sRing);
+        const uint64_t q_desc = sdesc_kmajor_sw128(smem_u32(sQ));
+        const uint64_t k_desc0 = sdesc_kmajor_sw128(ring_base);
+        const uint64_t v_desc0 = sdesc_mnmajor_sw128(ring_base, CHUNK_BYTES);
+        for (int j = 0; j <= n && ok; ++j) {
+          if (j >= 1) {
+            // O += P(j-1) V(j-1): keys 0..63 as soon as their half of P is written
+            if (!mbar_wait(p_half, (j - 1) & 1, s_abort, p.status, p.wait_ns) ||
+                !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t vd = v_desc0 + ((stage * TILE_BYTES) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
+                          (j > 1 || kk > 0) ? 1u : 0u);
+            if (!mbar_wait(p_full, (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 4; kk < 8; ++kk)
+              mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O, 1u);
+            mma_commit(&kv_empty[stage]);
+            if (j == n) mma_commit(o_final);
+            if (++stage == NSTAGE) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+          if (j < n) {
+            // S = Q K(j)^T into the S / P columns
+            if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kd = k_desc0 + ((stage * TILE_BYTES) >> 4);
+#pragma unroll
+            for (int c = 0; c < NCHUNK; ++c)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t off = (c * CHUNK_BYTES + kk * 32) >> 4;
+                mma_bf16_ss(tm_s, q_desc + off, kd + off, IDESC_S, (c | kk) != 0);
+              }
+            mma_commit(&kv_empty[stage]);
+            mma_commit(s_full);
+            if (++stage == NSTAGE) {
+              stage = 0;
+              phase ^= 1;
+            }
+          }
+        }
+        mma_commit(drain);
+        mbar_wait_drain(drain, 0);
+      }
     }
-  } else if (warp >= 4) {
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 160;\n" ::: "memory");
     // ------------------------------------------------------------ softmax + epilogue
     const int quad = warp & 3;
     const int r = quad * 32 + lane;

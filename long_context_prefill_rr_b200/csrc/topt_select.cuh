@@ -1,7 +1,7 @@
 // Top-tau selection of one block row by one warp (RRAttention "adaptive Top-tau selection";
 // the XAttention review, section 3, defines the rule as find_blocks: the smallest set of
-// blocks whose summed probability reaches tau). Shared by the standalone select kernel and the
-// estimate kernel's fused select. With masses a[0..I]:
+// blocks whose summed probability reaches tau), run by the standalone select kernel on one
+// row per warp. With masses a[0..I]:
 //
 //   sort J by a descending (ties: smaller J first), keep the shortest prefix whose running
 //   sum reaches tau * sum(a) (inclusive), add the diagonal J = I, emit ascending.
