@@ -725,7 +725,7 @@ def run_search_study(args):
 
 
 # bump when the attention kernel changes, so stale ncu traffic is not reported
-KERNEL_REV = "attn-v7-nreg"
+KERNEL_REV = "attn-v8-regs"
 
 
 def main(argv=None):

@@ -14,13 +14,15 @@
 //                the rest is), then S = Q K(j)^T into the same TMEM columns. It counts the
 //                item's valid tiles up front, so its issue loop reads no global memory;
 //   warp 2       TMEM allocation: S / P (128 columns) | O (d columns);
-//   warps 4-7    softmax: one thread per query row reads its 128 logits from TMEM, masks the
-//                diagonal block, keeps a running max (O is rescaled in TMEM, before any P of the
-//                tile is published, only when the max grows by more than 2^8, decided per warp)
-//                and running sum of the bf16-rounded weights, writes P as bf16 back over S in
-//                two halves, and at the end normalises O and stores the bf16 row.
+//   warps 4-7    softmax: one thread per query row reads its 128 logits from TMEM once into
+//                registers, masks the diagonal block, keeps a running max (O is rescaled in
+//                TMEM, before any P of the tile is published, only when the max grows by more
+//                than 2^8, decided per warp) and running sum of the bf16-rounded weights, writes
+//                P as bf16 back over S 16 keys at a time (keys 0..63 published first), and at
+//                the end normalises O and stores the bf16 row.
 // The first warpgroup (warps 0-3) runs with 96 registers a thread and the softmax warpgroup
-// with 160 (setmaxnreg), out of the 128 a thread the CTA is launched with.
+// with 160 (setmaxnreg), out of the 128 a thread the CTA is launched with; the 160 hold the
+// row's 128 logits.
 // Because the S / P columns are reused every tile, S(j) completing implies that the previous
 // P V product completed (MMAs complete in issue order), so O is stable whenever the softmax
 // runs. The kept list is read by every role with the same validity rule (0 <= J <= I, strictly
@@ -350,26 +352,24 @@ __global__ void __launch_bounds__(256, 2)
       }
       tc_fence_after();
       const bool diag = (J == I);   // diagonal block: key c is visible to query r iff c <= r
-      // pass 1: row max over the 128 logits, 64 columns at a time
+      // one read of the 128 logits; they stay in registers for the max and for P
+      float u[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(s_cols + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&u[c * 32]));
+      tmem_ld_wait();
+      if (diag) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c > r) u[c] = NEG_INF;
+      }
       float mx[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        float u[64];
-        tmem_ld32(s_cols + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tmem_ld32(s_cols + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_ld_wait();
-        if (diag) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (hh * 64 + c > r) u[c] = NEG_INF;
-        }
-#pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          mx[0] = fmax3(mx[0], u[c], u[c + 1]);
-          mx[1] = fmax3(mx[1], u[c + 2], u[c + 3]);
-          mx[2] = fmax3(mx[2], u[c + 4], u[c + 5]);
-          mx[3] = fmax3(mx[3], u[c + 6], u[c + 7]);
-        }
+      for (int c = 0; c < 128; c += 8) {
+        mx[0] = fmax3(mx[0], u[c], u[c + 1]);
+        mx[1] = fmax3(mx[1], u[c + 2], u[c + 3]);
+        mx[2] = fmax3(mx[2], u[c + 4], u[c + 5]);
+        mx[3] = fmax3(mx[3], u[c + 6], u[c + 7]);
       }
       const float tmax = fmax3(fmaxf(mx[0], mx[1]), mx[2], mx[3]) * sl2;
       float alpha = 1.f;
@@ -386,43 +386,38 @@ __global__ void __launch_bounds__(256, 2)
       }
       if (rescale) {
         // O is final for the previous tile (S(t) completing implies it); rescaled before any
-        // P of this tile is published
+        // P of this tile is published, 8 columns at a time (the logits hold the registers)
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(o_cols + c * 32, o);
+        for (int c = 0; c < D / 8; ++c) {
+          uint32_t o[8];
+          tmem_ld8(o_cols + c * 8, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-          tmem_st32(o_cols + c * 32, o);
+          for (int q = 0; q < 8; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+          tmem_st8(o_cols + c * 8, o);
         }
       }
-      // pass 2: P = 2^(u * scale_log2 - m) in bf16, written over S in two halves
+      // P = 2^(u * scale_log2 - m) in bf16, written over S 16 keys at a time (S is all in
+      // registers); keys 0..63 are published as soon as they are written
       const uint64_t negm = f2_pack(-m_run, -m_run);
-#pragma unroll 1
-      for (int hh = 0; hh < 2; ++hh) {
-        float u[64];
-        tmem_ld32(s_cols + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-        tmem_ld32(s_cols + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-        tmem_ld_wait();
-        if (diag) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (hh * 64 + c > r) u[c] = NEG_INF;
-        }
-        uint32_t pk[32];
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t pk[8];
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          const uint64_t xy = ffma2(f2_pack(u[2 * q], u[2 * q + 1]), sl2x2, negm);
+        for (int q = 0; q < 8; ++q) {
+          const int k = ch * 16 + 2 * q;
+          const uint64_t xy = ffma2(f2_pack(u[k], u[k + 1]), sl2x2, negm);
           pk[q] = pack_bf16x2(fast_exp2(f2_lo(xy)), fast_exp2(f2_hi(xy)));
           // the row sum takes the bf16 weights that P V uses, so O / l stays a convex
           // combination of the V rows (one dominant weight is no longer off by its rounding)
           add_bf16x2_to_f32(lsum[(2 * q) & 7], lsum[(2 * q + 1) & 7], pk[q]);
         }
-        tmem_st32(s_cols + hh * 32, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(hh == 0 ? p_half : p_full);
+        tmem_st8(s_cols + ch * 8, pk);
+        if (ch == 3 || ch == 7) {
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(ch == 3 ? p_half : p_full);
+        }
       }
     }
     __nv_bfloat16 *orow = p.out + (static_cast<int64_t>(bh) * p.L + I * 128 + r) * D;
