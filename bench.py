@@ -91,7 +91,12 @@ class ClockSampler:
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
                ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
-               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               # a clock set by an application or a user (a leftover lock) shows up here
+               ("applications_clocks_setting", "nvmlClocksEventReasonApplicationsClocksSetting"),
+               ("user_defined_clocks", "nvmlClocksEventReasonUserDefinedClocks"),
+               ("sync_boost", "nvmlClocksEventReasonSyncBoost"),
+               ("display_clock_setting", "nvmlClocksEventReasonDisplayClockSetting"))
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -117,7 +122,7 @@ class ClockSampler:
         import threading
         try:
             nv, h = self._nvml_handle()
-            bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS]
+            bits = [(name, getattr(nv, attr)) for name, attr in self.REASONS if hasattr(nv, attr)]
             mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
             self._stop = threading.Event()
 
