@@ -565,8 +565,8 @@ def run_gpu(args, w):
             "phases_ms": {"estimate_select": es_avg, "sparse_attn": att_avg},
             "phases_ms_spread": {"estimate_select": spread(es_ms), "sparse_attn": spread(att_ms),
                                  "step": spread([a + b for a, b in zip(es_ms, att_ms)])},
-            "phases_note": "estimate and select are one call (rra_estimate_select: pooled keys, estimate, select kernels); "
-                           "the pooled-key kernel is counted with them",
+            "phases_note": "estimate and select are one call (rra_estimate_select: the pooled-key, "
+                           "estimate and select kernels)",
             "density": density,
             "density_per_head": head_density(cnt_host),
             "attn_tflops": achieved, "attn_tflops_executed": executed / (att_avg * 1e-3) / 1e12,

@@ -128,10 +128,11 @@ rra_status rra_prefill(const rra_params *p, const void *q, const void *k, const 
  * copies run asynchronously. q_dev, k_dev, v_dev, out_dev are device staging buffers of the same
  * sizes, kept_idx / kept_cnt device outputs as in rra_prefill; the masses stay in the workspace,
  * which must hold rra_workspace_bytes(p).
- * The problem is cut into up to 16 chunks. With batch == 1 a chunk is a group of query heads
- * within one KV head, or whole KV heads when there are more than 16; the KV head's K and V are
- * copied with its first group. Otherwise a chunk is a group of batch rows. Each chunk is an independent sub-problem, because every
- * step is per (batch row, head); a chunk of heads runs with the round-robin shift advanced by its
+ * The problem is cut into up to 32 chunks. With batch == 1 a chunk is a group of query heads
+ * within one KV head, or whole KV heads when there are more than 32; the KV head's K and V are
+ * copied with its first group. Otherwise a chunk is a group of batch rows. Each chunk is an
+ * independent sub-problem, because every step is per (batch row, head); a chunk of heads runs
+ * with the round-robin shift advanced by its
  * first query head, so every head samples the offset it would sample in the whole problem, and
  * the results equal rra_prefill's. Chunk c's host-to-device copies run on an internal stream,
  * its estimate, select and attention on `stream` once they have landed, and its output copy on

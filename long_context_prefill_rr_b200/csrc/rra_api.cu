@@ -156,7 +156,7 @@ rra_status run_prefill(const Geometry &g, const void *q, const void *k, const vo
 }
 
 // Streams and events of rra_prefill_host, created once per device.
-constexpr int kMaxHostChunks = 16;
+constexpr int kMaxHostChunks = 32;
 struct HostPipe {
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t start = nullptr, end = nullptr;

@@ -9,9 +9,10 @@
 // No sort. With keys u_J = bits(a_J) (order-preserving for a >= 0) the cut value is v* = the
 // largest key with S(v*) = sum_{u_J >= v*} a_J >= tau * total, found by a bisection over the
 // key space up to the row's largest key, which stops as soon as one key is left in the interval
-// (at most 32 steps; about log2 of the row length in practice). Every block with a larger key is in the prefix; of the blocks tied at v*,
-// the first c in ascending J are, with c the smallest count that lifts the fp64 running sum to
-// the target. Ballots then compact the kept set in ascending order.
+// (at most 32 steps; about log2 of the row length in practice). Every block with a larger key
+// is in the prefix; of the blocks tied at v*, the first c in ascending J are, with c the
+// smallest count that lifts the fp64 running sum to the target. Ballots then compact the kept
+// set in ascending order.
 //
 // The decisions are the ones fp64 arithmetic gives: each bisection step first sums in fp32 and
 // falls back to an fp64 sum only when the fp32 sum lies within a margin of the target that

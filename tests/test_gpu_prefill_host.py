@@ -1,10 +1,11 @@
 """rra_prefill_host: host buffers in and out, chunked so that the copies overlap the compute.
 The chunks are independent sub-problems: query-head groups within a KV head, whole KV heads when
-there are more than 16, or batch rows. A chunk of heads runs with the round-robin shift advanced
-by its first head (the sampled offset rotates across heads: RRAttention abstract). Its kept lists
-and output are compared with the fp64 oracle run on the global heads and shift (kept lists of
-every row under the boundary rule, output rows sampled), and must equal rra_prefill's on the
-same inputs bit for bit. The cases cover each kind of chunk."""
+there are more than 32 (the mha48 case), or batch rows. A chunk of heads runs with the
+round-robin shift advanced by its first head (the sampled offset rotates across heads:
+RRAttention abstract). Its kept lists and output are compared with the fp64 oracle run on the
+global heads and shift (kept lists of every row under the boundary rule, output rows sampled),
+and must equal rra_prefill's on the same inputs bit for bit. The cases cover each kind of
+chunk."""
 import numpy as np
 import pytest
 import torch
@@ -20,7 +21,7 @@ CASES = {
     "llama8k": (wl.WORKLOADS["llama8k"], 1),
     "tiny_batch3": (wl.WORKLOADS["tiny"].with_(heads_kv=2, shift=3), 3),
     "video_short": (wl.WORKLOADS["video64k"].with_(seqlen=4096), 1),
-    "tiny_mha32": (wl.WORKLOADS["tiny"].with_(heads_q=32, heads_kv=32, shift=1), 1),
+    "tiny_mha48": (wl.WORKLOADS["tiny"].with_(heads_q=48, heads_kv=48, shift=1), 1),
 }
 
 
