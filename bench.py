@@ -5,7 +5,8 @@
 One step = one attention layer's prefill: pooled-key estimate, Top-tau select and block-sparse
 attention (rra_estimate, rra_select, rra_sparse_attn through the C ABI) on the seeded
 Llama-3.1-8B-like layer at 128K tokens (b1, 32 Q / 8 KV heads, d 128, B 128, S 8, tau 0.9).
-Inputs (2.7 GB) are larger than L2, so no flush is needed between steps. With N > 1 (torchrun)
+Inputs (1.61 GB at 128K) are larger than L2, so no flush is needed between steps; workloads whose
+inputs fit within twice the L2 size get an L2 flush before every timed step. With N > 1 (torchrun)
 every rank runs an independent replica of the layer (default), or with --shard heads its share
 of the KV-head groups of one layer (no exchange between ranks); the time is the max over ranks.
 
@@ -53,8 +54,31 @@ def _workload_desc(w: wl.Workload, parallelism: str = "replicas") -> dict:
             if w.kind == "llama" else w.kind,
             "global_batch": w.batch, "seq_len": w.seqlen, "heads_q": w.heads_q,
             "heads_kv": w.heads_kv, "head_dim": w.head_dim, "block": w.block, "stride": w.stride,
-            "tau": w.tau, "parallelism": parallelism, "l2": "inputs (2.7 GB) larger than L2"
-            if w.seqlen >= 32768 else "L2 flushed between steps"}
+            "tau": w.tau, "parallelism": parallelism, "l2": _l2_note(w)}
+
+
+def _input_bytes(w: wl.Workload) -> int:
+    """Q, K and V of the layer in bytes (bf16)."""
+    return 2 * w.batch * w.seqlen * w.head_dim * (w.heads_q + 2 * w.heads_kv)
+
+
+def _l2_bytes() -> int:
+    import torch
+    if torch.cuda.is_available():
+        return int(torch.cuda.get_device_properties(0).L2_cache_size)
+    return 126 << 20
+
+
+def _needs_flush(w: wl.Workload) -> bool:
+    """Inputs under twice the L2 size could be served from L2 across steps: flush between them."""
+    return _input_bytes(w) < 2 * _l2_bytes()
+
+
+def _l2_note(w: wl.Workload) -> str:
+    if _needs_flush(w):
+        return (f"inputs ({_input_bytes(w) / 1e9:.2f} GB) within 2x L2: L2 flushed between steps "
+                f"by writing {2 * _l2_bytes() >> 20} MiB (outside the per-step events)")
+    return f"inputs ({_input_bytes(w) / 1e9:.2f} GB) larger than 2x L2: no flush between steps"
 
 
 def attention_flops(kept_idx: np.ndarray, kept_cnt: np.ndarray, block: int, d: int):
@@ -476,12 +500,16 @@ def run_gpu(args, w):
         raise RuntimeError(f"device status {raw:#x} after warm-up")
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    flush = _needs_flush(w)
+    scrub = torch.empty(2 * _l2_bytes(), dtype=torch.uint8, device=dev) if flush else None
     if ws_n > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local) as clocks:
         start.record(stream)
         for s in range(args.steps):
+            if flush:
+                scrub.fill_(s & 0xFF)   # evicts the inputs from L2 before every timed step
             step(events[s])
         stop.record(stream)
         torch.cuda.synchronize(dev)
@@ -508,7 +536,8 @@ def run_gpu(args, w):
     torch.cuda.synchronize(dev)
     e2e_ms = e_start.elapsed_time(e_stop) / e_steps
 
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
+    ev_step_ms = float(np.mean(es_ms)) + float(np.mean(att_ms))
+    total_ms, e2e_ms, ev_step_ms = max_over_ranks([total_ms, e2e_ms, ev_step_ms], dev)
     cnt_host = cnt.cpu().numpy()
     idx_host = idx.cpu().numpy()
     useful, executed, n_kept = attention_flops(idx_host, cnt_host, w.block, w.head_dim)
@@ -536,7 +565,12 @@ def run_gpu(args, w):
                      + p.batch * p.heads_q * nb * (nb + 1) // 2 * 4)           # masses out
         sel_bytes = (p.batch * p.heads_q * nb * (nb + 1) // 2 * 4 + n_kept * 4 +
                      p.batch * p.heads_q * nb * 4)
-        ms_per_step = total_ms / args.steps
+        # with L2 flushes between the steps, a step's time is its own events' span (the flush
+        # sits outside it); otherwise the whole region over the steps
+        if flush:
+            ms_per_step = ev_step_ms
+        else:
+            ms_per_step = total_ms / args.steps
         # ms per layer of the whole job: replicas finish ws_n layers per step, head shards one
         value = ms_per_step if sharded else ms_per_step / ws_n
         cpu = None
