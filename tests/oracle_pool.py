@@ -58,6 +58,51 @@ def masses_full(q_bits, k_bits, batch, heads_q, heads_kv, seqlen, block, stride,
     return dict(zip(keys, res))
 
 
+def head_xattn_masses(args):
+    """fp64 XAttention (antidiagonal) masses of every block row of one (batch, head)."""
+    q_bits, k_bits, nb, block, stride, scale = args
+    q = wl.bf16_bits_to_f64(q_bits)
+    k = wl.bf16_bits_to_f64(k_bits)
+    out = np.empty(orc.tri_offset(nb), dtype=np.float64)
+    for I in range(nb):
+        out[orc.tri_offset(I):orc.tri_offset(I + 1)] = orc.xattn_estimate_block_row(
+            q, k, I, block, stride, scale)
+    return out
+
+
+def _pool_map(fn, tasks, workers):
+    """fn over tasks, serially or on spawned processes with one BLAS thread each."""
+    if workers is None:
+        workers = max(1, min(len(tasks), len(os.sched_getaffinity(0))))
+    if workers == 1 or len(tasks) <= 1:
+        return [fn(t) for t in tasks]
+    names = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+    saved = {v: os.environ.get(v) for v in names}
+    for v in names:
+        os.environ[v] = "1"
+    try:
+        ctx = multiprocessing.get_context("spawn")
+        with concurrent.futures.ProcessPoolExecutor(workers, mp_context=ctx) as ex:
+            return list(ex.map(fn, tasks))
+    finally:
+        for v, old in saved.items():
+            if old is None:
+                os.environ.pop(v, None)
+            else:
+                os.environ[v] = old
+
+
+def xattn_masses_full(q_bits, k_bits, batch, heads_q, heads_kv, seqlen, block, stride, scale,
+                      workers=None) -> dict:
+    """{(b, h): XAttention masses of every block row} for every (b, h)."""
+    nb = seqlen // block
+    keys = [(b, h) for b in range(batch) for h in range(heads_q)]
+    tasks = [(np.ascontiguousarray(q_bits[b, h]),
+              np.ascontiguousarray(k_bits[b, orc.kv_head(h, heads_q, heads_kv)]),
+              nb, block, stride, scale) for b, h in keys]
+    return dict(zip(keys, _pool_map(head_xattn_masses, tasks, workers)))
+
+
 def head_attention_errors(args):
     """Oracle attention of every query block of one (batch, head) on the GPU's kept lists,
     compared with the GPU's output rows: (max |gpu - ref|, sum (gpu - ref)^2, sum ref^2)."""

@@ -1,5 +1,6 @@
 """GPU parity of the XAttention antidiagonal estimator (rra_estimate_xattn) against the fp64
-oracle, and of the selection that follows it."""
+oracle, and of the selection that follows it: in full on Tiny variants and on every block row
+of the Llama-like layer at 8K and 32K."""
 import numpy as np
 import pytest
 import torch
@@ -46,18 +47,28 @@ def test_xattn_full_parity(cuda_device, label, over):
     print(f"[xattn {label}] mass_err={err:.3g}")
 
 
-@pytest.mark.parametrize("name,n_rows", [("llama8k", 96), ("llama32k", 32)])
-def test_xattn_sampled_parity(cuda_device, name, n_rows):
+@pytest.mark.parametrize("name", ["llama8k", "llama32k"])
+def test_xattn_parity_at_length(cuda_device, name):
+    """Every mass of every head against the fp64 oracle (one head per spawned process), the
+    select on those masses bit-exact against the oracle's select on the same fp32 masses, and
+    the kept lists against the oracle's own lists outside the boundary rule."""
+    import oracle_pool
     w, p = par.workload_params(wl.WORKLOADS[name])
     qb, kb, _ = wl.make_workload(w)
     gpu = _run(p, qb, kb)
-    qc, kc = par.HeadCache(qb), par.HeadCache(kb)
-    scale = par.resolved_scale(p)
-    err = 0.0
-    for b, h, I in par.sample_rows(p, n_rows, seed=7):
-        kv = orc.kv_head(h, w.heads_q, w.heads_kv)
-        want = orc.xattn_estimate_block_row(qc(b, h), kc(b, kv), I, w.block, w.stride, scale)
-        got = gpu[b, h, orc.tri_offset(I):orc.tri_offset(I + 1)]
-        err = max(err, float(np.abs(got - want).max()))
+    full = oracle_pool.xattn_masses_full(qb, kb, p.batch, p.heads_q, p.heads_kv, p.seqlen,
+                                         p.block, p.stride, par.resolved_scale(p))
+    err = max(float(np.abs(gpu[b, h] - a).max()) for (b, h), a in full.items())
     assert err <= par.MASS_ATOL, err
-    print(f"[xattn {name}] mass_err={err:.3g}")
+    nb = w.seqlen // w.block
+    sh = native.shapes(p)
+    idx = torch.empty(sh["kept_idx"], dtype=torch.int32, device="cuda")
+    cnt = torch.empty(sh["kept_cnt"], dtype=torch.int32, device="cuda")
+    native.select(p, torch.from_numpy(gpu).cuda(), idx, cnt)
+    res = dict(mass=gpu, idx=idx.cpu().numpy(), cnt=cnt.cpu().numpy())
+    assert par.select_on_gpu_masses_exact(res, w.tau, nb), "select on GPU masses"
+    rows = par.mass_rows(full, nb)
+    mism, exc, n = par.compare_select_rows(res, rows, w.tau)
+    assert not mism, mism[:5]
+    par.record(f"xattn_{name}", mass_rows=len(rows), mass_max_err=err, list_rows=n,
+               list_mismatch_excused=len(exc), boundary_rows=par.boundary_count(rows, w.tau))
