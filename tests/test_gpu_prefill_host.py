@@ -3,7 +3,7 @@ The chunks are independent sub-problems: query-head groups within a KV head, who
 there are more than 32 (the mha48 case), or batch rows. A chunk of heads runs with the
 round-robin shift advanced by its first head (the sampled offset rotates across heads:
 RRAttention abstract). Its kept lists and output are compared with the fp64 oracle run on the
-global heads and shift (kept lists of every row under the boundary rule, output rows sampled),
+global heads and shift (kept lists of every row under the boundary rule, every output row),
 and must equal rra_prefill's on the same inputs bit for bit. The cases cover each kind of
 chunk."""
 import numpy as np
@@ -63,10 +63,10 @@ def test_prefill_host_equals_prefill(cuda_device, name):
     full = par.oracle_masses_full(qb, kb, p)
     mism, exc, n = par.compare_select_rows(got, par.mass_rows(full, nb), w.tau)
     assert not mism, f"{name}: kept-list mismatches outside the boundary rule: {mism[:5]}"
-    qc, kc, vc = par.HeadCache(qb), par.HeadCache(kb), par.HeadCache(vb)
-    rows = par.sample_rows(p, 24, seed=7)
-    ref_rows = par.oracle_attention_rows(qc, kc, vc, p, got["idx"], got["cnt"], rows)
-    ma, rr = par.attention_rows_errors(got["out"], ref_rows)
+    import oracle_pool
+    ma, rr, n_attn = oracle_pool.attention_errors_full(
+        qb, kb, vb, got["out"], got["idx"], got["cnt"], p.heads_q, p.heads_kv, p.block,
+        par.resolved_scale(p))
     assert ma <= par.ATTN_MAX_ABS and rr <= par.ATTN_REL_RMS, (name, ma, rr)
     par.record(f"prefill_host_{name}", list_rows=n, list_mismatch_excused=len(exc),
-               attn_rows=f"sampled {len(rows)}", attn_max_abs=ma, attn_rel_rms=rr)
+               attn_rows=f"all {n_attn}", attn_max_abs=ma, attn_rel_rms=rr)
