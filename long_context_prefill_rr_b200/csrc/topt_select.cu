@@ -1,14 +1,15 @@
 // Standalone Top-tau select kernel: one warp per (batch, head, block row I) runs the row
 // select of topt_select.cuh on masses read from global memory. Rows of up to 1024 blocks are
 // held in registers, in a variant specialised to the row's chunk count; longer rows are re-read
-// from memory in every pass.
+// from memory in every pass. Three 256-thread blocks per SM (78 registers a thread, no spills):
+// each bisection step waits on a warp reduction, so more resident warps hide that latency.
 #include "common.cuh"
 #include "rra_internal.h"
 #include "topt_select.cuh"
 
 namespace rra {
 
-__global__ void __launch_bounds__(256) topt_select_kernel(const float *__restrict__ mass,
+__global__ void __launch_bounds__(256, 3) topt_select_kernel(const float *__restrict__ mass,
                                                           int32_t *__restrict__ kept_idx,
                                                           int32_t *__restrict__ kept_cnt,
                                                           int64_t rows, int nb, int64_t tri,
