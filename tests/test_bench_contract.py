@@ -63,3 +63,18 @@ def test_workload_overrides_reach_the_config():
     d = json.loads(r.stdout.strip().splitlines()[-1])
     assert d["config"]["stride"] == 16 and d["config"]["tau"] == 0.95
     assert "S16" in d["config"]["workload"] and "tau0.95" in d["config"]["workload"]
+
+
+def test_l2_flush_applies_where_inputs_fit_twice_the_l2(monkeypatch):
+    """Layers whose Q, K and V fit within twice the L2 are flushed before each timed step, and
+    the config says which case applies with the real input size."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_context_prefill_rr_b200 import workloads as wl
+    monkeypatch.setattr(bench, "_l2_bytes", lambda: 126 << 20)
+    w8, w32, w128 = (wl.WORKLOADS[n] for n in ("llama8k", "llama32k", "llama128k"))
+    assert bench._input_bytes(w128) == 2 * 131072 * 128 * (32 + 16)
+    assert bench._needs_flush(w8) and not bench._needs_flush(w32)
+    assert not bench._needs_flush(w128) and not bench._needs_flush(wl.WORKLOADS["video64k"])
+    assert "flushed" in bench._workload_desc(w8)["l2"] and "0.10 GB" in bench._l2_note(w8)
+    assert "no flush" in bench._workload_desc(w128)["l2"] and "1.61 GB" in bench._l2_note(w128)
