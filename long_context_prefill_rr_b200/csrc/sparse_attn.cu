@@ -3,7 +3,7 @@
 // digest; online softmax as in FlashAttention / FlashAttention-2), GQA head mapping.
 //
 // One CTA runs one work item: query block I of one head. Its footprint (256 threads, 256 TMEM
-// columns, about 97 KB of shared memory) lets two CTAs share an SM, so the tensor core works on
+// columns, about 99 KB of shared memory) lets two CTAs share an SM, so the tensor core works on
 // one CTA's tile while the other CTA's softmax runs, and one CTA's set-up and epilogue overlap
 // the other's work. Grid order is longest-first (I descending), by KV-head chunk when K and V
 // exceed L2 (see attn_item). Roles:
