@@ -764,7 +764,7 @@ def run_search_study(args):
 
 
 # bump when the attention kernel changes, so stale ncu traffic is not reported
-KERNEL_REV = "attn-v8-regs"
+KERNEL_REV = "attn-v9-pq4"
 
 
 def main(argv=None):

@@ -10,15 +10,15 @@
 //   warp 0       TMA producer: the Q tile, then V(j-1), K(j) through a two-tile ring, in the
 //                order the MMA warp consumes them;
 //   warp 1       MMA issuer (one thread): O += P(j-1) V(j-1) with P read from TMEM (tcgen05
-//                "TS" form; keys 0..63 as soon as that half of P is written, keys 64..127 when
-//                the rest is), then S = Q K(j)^T into the same TMEM columns. It counts the
+//                "TS" form; 32 keys at a time, as soon as that quarter of P is written), then
+//                S = Q K(j)^T into the same TMEM columns. It counts the
 //                item's valid tiles up front, so its issue loop reads no global memory;
 //   warp 2       TMEM allocation: S / P (128 columns) | O (d columns);
 //   warps 4-7    softmax: one thread per query row reads its 128 logits from TMEM once into
 //                registers, masks the diagonal block, keeps a running max (O is rescaled in
 //                TMEM, before any P of the tile is published, only when the max grows by more
 //                than 2^8, decided per warp) and running sum of the bf16-rounded weights, writes
-//                P as bf16 back over S 16 keys at a time (keys 0..63 published first), and at
+//                P as bf16 back over S 16 keys at a time (published 32 keys at a time), and at
 //                the end normalises O and stores the bf16 row.
 // The first warpgroup (warps 0-3) runs with 96 registers a thread and the softmax warpgroup
 // with 160 (setmaxnreg), out of the 128 a thread the CTA is launched with; the 160 hold the
@@ -161,9 +161,8 @@ __global__ void __launch_bounds__(256, 2)
   uint64_t *kv_full = bars + 1;                     // [NSTAGE]
   uint64_t *kv_empty = kv_full + NSTAGE;            // [NSTAGE]
   uint64_t *s_full = kv_empty + NSTAGE;
-  uint64_t *p_full = s_full + 1;
-  uint64_t *p_half = p_full + 1;                    // P of keys 0..63 written
-  uint64_t *o_final = p_half + 1;
+  uint64_t *p_q = s_full + 1;                       // [4] P of keys 32q..32q+31 written
+  uint64_t *o_final = p_q + 4;
   uint64_t *drain = o_final + 1;
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
@@ -185,8 +184,7 @@ __global__ void __launch_bounds__(256, 2)
       mbar_init(&kv_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
-    mbar_init(p_half, 128);
+    for (int i = 0; i < 4; ++i) mbar_init(&p_q[i], 128);
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *s_abort = 0;
@@ -274,26 +272,24 @@ __global__ void __launch_bounds__(256, 2)
         const uint64_t v_desc0 = sdesc_mnmajor_sw128(ring_base, CHUNK_BYTES);
         for (int j = 0; j <= n && ok; ++j) {
           if (j >= 1) {
-            // O += P(j-1) V(j-1): keys 0..63 as soon as their half of P is written
-            if (!mbar_wait(p_half, (j - 1) & 1, s_abort, p.status, p.wait_ns) ||
-                !mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
+            // O += P(j-1) V(j-1): 32 keys at a time, as soon as that quarter of P is written
+            if (!mbar_wait(&kv_full[stage], phase, s_abort, p.status, p.wait_ns)) {
               ok = false;
               break;
             }
-            tc_fence_after();
             const uint64_t vd = v_desc0 + ((stage * TILE_BYTES) >> 4);
+            for (int qq = 0; qq < 4 && ok; ++qq) {
+              if (!mbar_wait(&p_q[qq], (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
-                          (j > 1 || kk > 0) ? 1u : 0u);
-            if (!mbar_wait(p_full, (j - 1) & 1, s_abort, p.status, p.wait_ns)) {
-              ok = false;
-              break;
+              for (int kk = 2 * qq; kk < 2 * qq + 2; ++kk)
+                mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O,
+                            (j > 1 || kk > 0) ? 1u : 0u);
             }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 4; kk < 8; ++kk)
-              mma_bf16_ts(tm_o, tm_s + kk * 8, vd + kk * (2048 >> 4), IDESC_O, 1u);
+            if (!ok) break;
             mma_commit(&kv_empty[stage]);
             if (j == n) mma_commit(o_final);
             if (++stage == NSTAGE) {
@@ -398,7 +394,7 @@ __global__ void __launch_bounds__(256, 2)
         }
       }
       // P = 2^(u * scale_log2 - m) in bf16, written over S 16 keys at a time (S is all in
-      // registers); keys 0..63 are published as soon as they are written
+      // registers); each 32 keys are published as soon as they are written
       const uint64_t negm = f2_pack(-m_run, -m_run);
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
@@ -413,10 +409,10 @@ __global__ void __launch_bounds__(256, 2)
           add_bf16x2_to_f32(lsum[(2 * q) & 7], lsum[(2 * q + 1) & 7], pk[q]);
         }
         tmem_st8(s_cols + ch * 8, pk);
-        if (ch == 3 || ch == 7) {
+        if (ch & 1) {
           tmem_st_wait();
           tc_fence_before();
-          mbar_arrive(ch == 3 ? p_half : p_full);
+          mbar_arrive(&p_q[ch >> 1]);
         }
       }
     }
@@ -460,7 +456,7 @@ static cudaError_t launch_attn_t(const CUtensorMap &mq, const CUtensorMap &mk,
                                   cudaStream_t stream) {
   constexpr size_t TILE = static_cast<size_t>(D / 64) * 128 * 128;
   constexpr int NSTAGE = (D == 128) ? 2 : 4;
-  const size_t smem = 1024 + TILE * (1 + NSTAGE) + (2 * NSTAGE + 6) * 8 + 16;
+  const size_t smem = 1024 + TILE * (1 + NSTAGE) + (2 * NSTAGE + 8) * 8 + 16;
   auto kern = bs_attn_fwd_kernel<D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
